@@ -1,0 +1,176 @@
+"""CPU fp64 oracle for exact softmax attention (forward and backward).
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this module: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It
+shares no code with the CUDA library and imports nothing from the package.
+
+What it computes, and where each step is stated:
+
+* Scores, probabilities, output -- "Flash attention and efficient attention",
+  section "The Standard Attention Problem": S = Q K^T, P = softmax(S / sqrt(d_k)),
+  O = P V.  The scale is an explicit argument (the pages fold 1/sqrt(d_k) into
+  the softmax; callers pass 1/sqrt(d) for that reading).
+* Safe softmax -- same page, "Derivation: Incremental Softmax", Step 1: the
+  row maximum is subtracted before exponentiating.  This oracle is the plain
+  two-pass form (max, then exp/sum); the tiled, online form that the GPU runs is
+  equal to it in exact arithmetic (page "FlashAttention paper", section
+  "Exact, not approximate").
+* Masks -- causal keeps keys j <= i ("FlashAttention" guide page, section
+  "Tiling through SRAM": causal masks change tiling, not the rule); the local
+  window keeps |i - j| <= w, which reproduces the N=6, w=3 matrix of the
+  "Flash attention and efficient attention" page, worked example
+  "Local Attention Window" (there w counts the token and one neighbour on each
+  side, i.e. half-width 1 here).
+* Saved softmax metadata -- the per-row natural-log logsumexp of the scaled,
+  masked scores, LSE_i = m_i + ln(sum_j exp(S_ij - m_i)).  The pages only call
+  it "a little softmax metadata" ("FlashAttention" guide page, "Tiling through
+  SRAM"); this is the plainest reading.
+* Backward -- the pages say only that S and P are recomputed from Q, K, V
+  ("Flash attention and efficient attention", section "Backward Pass:
+  Recomputation").  The formulas below are the textbook softmax Jacobian for
+  the loss L = sum(dO * O):
+      dV = P^T dO,  dP = dO V^T,  D_i = sum_j P_ij dP_ij,
+      dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+  D is taken from P and dP on purpose (not as rowsum(dO * O)).
+* GQA -- query head h reads kv head h // (H / Hkv); the gradients of a kv
+  head sum over its query heads.  The guide page only names grouped-query
+  attention, so this contiguous grouping is a reading.
+* Fully masked rows (impossible in the shipped workloads, where the diagonal
+  is always allowed) give O = 0, LSE = -inf and zero gradients.
+
+Implementation notes, none of which changes a value: rows are processed in
+blocks (each row's softmax is still computed over its whole key range at once),
+and with a causal or window mask only keys that can be allowed for a block are
+materialised; every other key contributes exactly zero.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = ["allowed", "attention_probs", "forward", "backward", "row_dot"]
+
+
+def allowed(rows: np.ndarray, cols: np.ndarray, causal: bool, window: int) -> np.ndarray:
+    """Boolean mask a[i, j]: may query ``rows[i]`` attend to key ``cols[j]``?
+
+    causal -> j <= i; window >= 0 -> |i - j| <= window; window = -1 -> no band.
+    """
+    r = np.asarray(rows)[:, None]
+    c = np.asarray(cols)[None, :]
+    ok = np.ones((r.shape[0], c.shape[1]), dtype=bool)
+    if causal:
+        ok &= c <= r
+    if window >= 0:
+        ok &= np.abs(r - c) <= window
+    return ok
+
+
+def _key_range(r0: int, r1: int, n: int, causal: bool, window: int) -> tuple[int, int]:
+    lo, hi = 0, n
+    if causal:
+        hi = min(hi, r1)
+    if window >= 0:
+        lo = max(lo, r0 - window)
+        hi = min(hi, r1 + window)
+    return lo, max(lo, hi)
+
+
+def _scores(q_rows, k_keys, scale, rows, keys, causal, window):
+    s = scale * (q_rows @ k_keys.T)
+    ok = allowed(rows, keys, causal, window)
+    s = np.where(ok, s, -np.inf)
+    return s, ok
+
+
+def attention_probs(q_rows, k_keys, scale, rows, keys, causal, window):
+    """Safe softmax of the masked, scaled scores of one head.
+
+    Returns (P, m, l): P[i, j] probabilities, m the row max of the scaled
+    scores, l = sum_j exp(S_ij - m_i).  Rows with no allowed key get P = 0,
+    m = -inf, l = 0.
+    """
+    s, ok = _scores(q_rows, k_keys, scale, rows, keys, causal, window)
+    m = s.max(axis=1) if s.shape[1] else np.full(s.shape[0], -np.inf)
+    dead = ~np.isfinite(m)
+    m_safe = np.where(dead, 0.0, m)
+    e = np.where(ok, np.exp(s - m_safe[:, None]), 0.0)
+    l = e.sum(axis=1)
+    p = np.where(l[:, None] > 0, e / np.where(l > 0, l, 1.0)[:, None], 0.0)
+    return p, m, l
+
+
+def _as64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # a torch tensor; upcast exactly from its dtype
+        x = x.detach().cpu().double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def _heads(q, k):
+    b, h, n, d = q.shape
+    hkv = k.shape[1]
+    if h % hkv:
+        raise ValueError("H must be a multiple of Hkv")
+    return b, h, hkv, n, d, h // hkv
+
+
+def forward(q, k, v, scale: float, causal: bool = False, window: int = -1,
+            heads=None, row_block: int = 2048):
+    """O [B,H,N,d] and LSE [B,H,N] in fp64.
+
+    q: [B,H,N,d]; k, v: [B,Hkv,N,d].  ``heads`` optionally restricts the work to
+    a list of (b, h) pairs; other heads are left as NaN.
+    """
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    b_, h_, _, n, d, g = _heads(q, k)
+    o = np.full(q.shape, np.nan)
+    lse = np.full(q.shape[:3], np.nan)
+    todo = heads if heads is not None else [(b, h) for b in range(b_) for h in range(h_)]
+    for b, h in todo:
+        kvh = h // g
+        for r0 in range(0, n, row_block):
+            r1 = min(n, r0 + row_block)
+            lo, hi = _key_range(r0, r1, n, causal, window)
+            rows, keys = np.arange(r0, r1), np.arange(lo, hi)
+            p, m, l = attention_probs(q[b, h, r0:r1], k[b, kvh, lo:hi], scale,
+                                      rows, keys, causal, window)
+            o[b, h, r0:r1] = p @ v[b, kvh, lo:hi]
+            with np.errstate(divide="ignore"):
+                lse[b, h, r0:r1] = np.where(l > 0, m + np.log(np.where(l > 0, l, 1.0)), -np.inf)
+    return o, lse
+
+
+def row_dot(p: np.ndarray, dp: np.ndarray) -> np.ndarray:
+    """D_i = sum_j P_ij dP_ij (the softmax-Jacobian row term)."""
+    return (p * dp).sum(axis=1)
+
+
+def backward(q, k, v, do, scale: float, causal: bool = False, window: int = -1,
+             heads=None, row_block: int = 2048):
+    """dQ [B,H,N,d], dK and dV [B,Hkv,N,d] of L = sum(dO * O), in fp64.
+
+    S and P are recomputed from Q and K (no saved forward state is used).
+    With ``heads`` only those (b, h) query heads contribute: dQ of other heads
+    is NaN and dK/dV hold only the listed heads' contributions.
+    """
+    q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
+    b_, h_, _, n, d, g = _heads(q, k)
+    dq = np.full(q.shape, np.nan)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    todo = heads if heads is not None else [(b, h) for b in range(b_) for h in range(h_)]
+    for b, h in todo:
+        kvh = h // g
+        for r0 in range(0, n, row_block):
+            r1 = min(n, r0 + row_block)
+            lo, hi = _key_range(r0, r1, n, causal, window)
+            rows, keys = np.arange(r0, r1), np.arange(lo, hi)
+            kk, vv = k[b, kvh, lo:hi], v[b, kvh, lo:hi]
+            qq, dd = q[b, h, r0:r1], do[b, h, r0:r1]
+            p, _, _ = attention_probs(qq, kk, scale, rows, keys, causal, window)
+            dv[b, kvh, lo:hi] += p.T @ dd
+            dp = dd @ vv.T
+            ds = p * (dp - row_dot(p, dp)[:, None])
+            dq[b, h, r0:r1] = scale * (ds @ kk)
+            dk[b, kvh, lo:hi] += scale * (ds.T @ qq)
+    return dq, dk, dv
