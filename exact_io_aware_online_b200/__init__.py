@@ -1,0 +1,130 @@
+"""Exact IO-aware online-softmax attention for B200 (sm_100a).
+
+The compute lives in ``libfa.so`` (CUDA kernels behind the C ABI of
+``include/fa.h``).  This package only marshals arguments: ``lib()`` loads the
+shared library with ctypes and the ``fwd`` / ``bwd`` helpers allocate outputs
+with PyTorch and pass raw device pointers and the current stream.  There is no
+CPU fallback: if the library is missing or a call fails, an error is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+__all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
+           "exported_names", "LIB_PATH", "HEADER_PATH"]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa.so")
+HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "fa.h")
+
+FA_BF16, FA_FP32 = 0, 1
+STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_MISALIGNED",
+          4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA", 6: "FA_ERR_TIMEOUT"}
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}" if what else STATUS.get(code, str(code)))
+
+
+def exported_names() -> list[str]:
+    """Function names declared in include/fa.h."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_]+\**\s+\**(fa_[a-z_0-9]+)\s*\(", text, re.M)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_online_b200._build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
+    L.fa_fwd.restype = i
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, i, vp]
+    L.fa_bwd.restype = i
+    L.fa_bwd_workspace_size.argtypes = [i, i, i, i, i]
+    L.fa_bwd_workspace_size.restype = sz
+    L.fa_last_device_status.argtypes = [vp]
+    L.fa_last_device_status.restype = i
+    L.fa_status_string.argtypes = [i]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_version.argtypes = []
+    L.fa_version.restype = i
+    _lib = L
+    return L
+
+
+# ---------------------------------------------------------------------------
+# torch-facing helpers (argument marshalling only)
+# ---------------------------------------------------------------------------
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float32:
+        return FA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream_ptr(device) -> int:
+    import torch
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise FAError(code, what)
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype_code: int) -> int:
+    return int(lib().fa_bwd_workspace_size(B, H, N, d, dtype_code))
+
+
+def fwd(q, k, v, scale: float | None = None, causal: bool = False, window: int = -1, out=None, lse=None):
+    """O, LSE = attention(q [B,H,N,d], k/v [B,Hkv,N,d]); outputs allocated if not given."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    code = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                        B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
+                        _stream_ptr(q.device))
+    _check(code, "fa_fwd")
+    return o, l
+
+
+def bwd(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = -1,
+        workspace=None, grads=None):
+    """dQ, dK, dV of sum(do * o); workspace and gradients allocated if not given."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    code_t = _dtype_code(q)
+    need = bwd_workspace_size(B, H, N, d, code_t)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    code = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                        dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
+                        B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), code_t,
+                        _stream_ptr(q.device))
+    _check(code, "fa_bwd")
+    return dq, dk, dv
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    import torch
+    return int(lib().fa_last_device_status(torch.cuda.current_stream(device).cuda_stream))

@@ -1,0 +1,464 @@
+// bwd_sm100.cuh -- bf16 attention backward on sm_100a tensor cores.
+//
+// The backward pass recomputes the scores and probabilities tile by tile from
+// Q, K and the saved logsumexp instead of reading an N x N matrix ("Flash
+// attention and efficient attention", section "Backward Pass: Recomputation";
+// "FlashAttention" guide page, "Tiling through SRAM").  The gradient formulas
+// are the softmax Jacobian for L = sum(dO * O):
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  D_i = dO_i . O_i,
+//   dK = scale dS^T Q,  dQ = scale dS K.
+//
+// Three kernels run on one stream:
+//   bwd_pre_kernel   D_i, LSE_i * log2(e) (+inf on padding rows) and a zeroed
+//                    fp32 dQ accumulator, all in the caller's workspace;
+//   bwd_sm100_kernel one CTA per (batch, kv head, 128-key tile): K_j and V_j
+//                    stay in shared memory while the CTA walks every query
+//                    tile (of every query head of the GQA group) that can see
+//                    them; dK_j and dV_j accumulate in TMEM and are written
+//                    once, dQ partial tiles are added into the accumulator;
+//   bwd_dq_kernel    dQ = bf16(scale * accumulator).
+//
+// Main-kernel roles (320 threads):
+//   warps 0-3  P / dS: one thread per key row (TMEM lanes 0-127)
+//   warps 4-7  dQ drain (one thread per query row of the dQ tile) and the
+//              final dK/dV epilogue (one thread per key row)
+//   warp 8     tcgen05.mma issuer and TMEM owner
+//   warp 9     TMA producer
+// The products are formed transposed (S^T = K Q^T, dP^T = V dO^T) so that P^T
+// and dS^T land in TMEM with one key row per lane and can be fed back, as
+// packed bf16, as the A operand of dV += P^T dO and dK += dS^T Q.  dS itself
+// (needed with queries as rows for dQ = dS K) is written to shared memory in
+// the MN-major layout the tensor core reads.
+// TMEM: S^T [0,128) (P^T packed over [0,64)), dP^T [128,256) (dS^T packed over
+// [128,192)), dV [256,256+D), dK [256+D,256+2D); the dQ tile takes [128,256)
+// for D = 128 (after dS^T has been consumed) and [384,448) for D = 64.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const float* lse;  // [B*H*N] from the forward
+  const void* o;     // bf16 [B*H*N*D]
+  const void* dout;  // bf16 [B*H*N*D]
+  float* lse2;       // workspace [B*H*Np]: lse*log2(e), +inf on rows >= N
+  float* Drow;       // workspace [B*H*Np]: D_i, 0 on rows >= N
+  float* dqacc;      // workspace [B*H*Np*D]
+  void* dq;          // bf16 [B*H*N*D]
+  int B, H, Hkv, N, Np, g;
+  float scale, scale_log2;
+  int causal, window;
+  int ntiles;  // Np / 128
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kChunks = D / 64;
+  static constexpr int kStages = (D == 128) ? 2 : 3;  // (Q, dO) tile pairs in flight
+  static constexpr int kDsBytes = 128 * 128 * 2;
+  static constexpr int kNumBars = 1 + 2 * kStages + 8;
+  static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + kStages * 2 * kTileBytes + kDsBytes + 8 * kNumBars + 16;
+  static constexpr bool kAliasDq = (D == 128);
+  static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
+  static constexpr uint32_t kColDQ = kAliasDq ? 128 : 256 + 2 * D;
+};
+
+// ---------------------------------------------------------------- preprocess
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(blockIdx.x) * 8 + warp;  // over B*H*Np
+  const size_t rows = static_cast<size_t>(p.B) * p.H * p.Np;
+  if (row >= rows) return;
+  const size_t bh = row / p.Np;
+  const int n = static_cast<int>(row % p.Np);
+  float4* acc = reinterpret_cast<float4*>(p.dqacc + row * D);
+  for (int x = lane; x < D / 4; x += 32) acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (n >= p.N) {
+    if (lane == 0) {
+      p.Drow[row] = 0.f;
+      p.lse2[row] = INFINITY;
+    }
+    return;
+  }
+  const size_t src = (bh * p.N + n) * D;
+  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(p.o) + src / 2;
+  const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(p.dout) + src / 2;
+  float s = 0.f;
+  for (int x = lane; x < D / 2; x += 32) {
+    const float2 a = __bfloat1622float2(o2[x]);
+    const float2 c = __bfloat1622float2(d2[x]);
+    s = fmaf(a.x, c.x, fmaf(a.y, c.y, s));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) {
+    p.Drow[row] = s;
+    p.lse2[row] = p.lse[bh * p.N + n] * 1.4426950408889634f;
+  }
+}
+
+// ---------------------------------------------------------------- dQ convert
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
+  const size_t i4 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // float4 index
+  const size_t total4 = static_cast<size_t>(p.B) * p.H * p.N * D / 4;
+  if (i4 >= total4) return;
+  const size_t e = i4 * 4;
+  const size_t row = e / D, col = e % D;
+  const size_t bh = row / p.N, n = row % p.N;
+  const float4 a = *reinterpret_cast<const float4*>(p.dqacc + (bh * p.Np + n) * D + col);
+  uint2 out;
+  out.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
+  out.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
+  *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + e) = out;
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(a)),
+               "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
+               : "memory");
+}
+
+// Writes 32 fp32 values of row r (columns c..c+31 of a D-wide row), converted to
+// bf16, into a 128-row tile staged in the TMA 128-byte-swizzled layout.
+__device__ __forceinline__ void stage_row32_bf16(uint8_t* tile, int r, int c, const uint32_t (&v)[32], float mul) {
+  const int chunk = c >> 6, u0 = (c & 63) >> 3;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint4 val;
+    val.x = pack_bf16x2(__uint_as_float(v[8 * u + 0]) * mul, __uint_as_float(v[8 * u + 1]) * mul);
+    val.y = pack_bf16x2(__uint_as_float(v[8 * u + 2]) * mul, __uint_as_float(v[8 * u + 3]) * mul);
+    val.z = pack_bf16x2(__uint_as_float(v[8 * u + 4]) * mul, __uint_as_float(v[8 * u + 5]) * mul);
+    val.w = pack_bf16x2(__uint_as_float(v[8 * u + 6]) * mul, __uint_as_float(v[8 * u + 7]) * mul);
+    *reinterpret_cast<uint4*>(tile + chunk * 16384 + r * 128 + (((u0 + u) ^ (r & 7)) << 4)) = val;
+  }
+}
+
+// ---------------------------------------------------------------- main kernel
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                     const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                     const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sK = base;
+  uint8_t* sV = base + C::kTileBytes;
+  uint8_t* sStage = base + 2 * C::kTileBytes;  // stage s: Q at +0, dO at +kTileBytes
+  uint8_t* sDS = sStage + C::kStages * 2 * C::kTileBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + C::kDsBytes);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = bars + 1 + C::kStages;
+  uint64_t* s_full = bars + 1 + 2 * C::kStages;
+  uint64_t* dp_full = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* ds_full = s_full + 3;
+  uint64_t* dq_full = s_full + 4;
+  uint64_t* dq_empty = s_full + 5;
+  uint64_t* kv_done = s_full + 6;
+  uint64_t* epi_bar = s_full + 7;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work unit: key tile j of kv head (b, kh); small j (most query tiles under a causal mask) first
+  const int BHkv = p.B * p.Hkv;
+  const int j = static_cast<int>(blockIdx.x) / BHkv;
+  const int bkv = static_cast<int>(blockIdx.x) % BHkv;
+  const int b = bkv / p.Hkv, kh = bkv % p.Hkv;
+  const int k0 = j * 128;
+  int ilo = 0, ihi = p.ntiles - 1;
+  if (p.causal) ilo = j;
+  if (p.window >= 0) {
+    ilo = max(ilo, max(0, k0 - p.window) / 128);
+    ihi = min(ihi, (k0 + 127 + p.window) / 128);
+  }
+  const int nq = ihi - ilo + 1;
+  const int total = nq * p.g;
+  auto q_tile = [&](int it) { return ilo + it % nq; };
+  auto q_head = [&](int it) { return b * p.H + kh * p.g + it / nq; };
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(ds_full, 128);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 128);
+    mbar_init(kv_done, 1);
+    mbar_init(epi_bar, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      prefetch_tmap(&tmdO);
+      mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, k0, bkv);
+        tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, k0, bkv);
+      }
+      int issued[C::kStages];
+#pragma unroll
+      for (int i = 0; i < C::kStages; ++i) issued[i] = 0;
+      for (int it = 0; it < total; ++it) {
+        const int s = it % C::kStages;
+        if (!mbar_wait(&q_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&q_full[s], 2 * C::kTileBytes);
+        const int row0 = q_tile(it) * 128, bh = q_head(it);
+        uint8_t* st = sStage + s * 2 * C::kTileBytes;
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
+          tma_load_3d(&tmdO, &q_full[s], st + C::kTileBytes + c * 16384, c * 64, row0, bh);
+        }
+        ++issued[s];
+      }
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(kv_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+      for (int s = 0; s < C::kStages; ++s)
+        if (issued[s] > 0)
+          while (!mbar_try_wait(smem_u32(&q_full[s]), (issued[s] - 1) & 1) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aSt = smem_u32(sStage), aDS = smem_u32(sDS);
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t kIdG = idesc_bf16_f32(128, D, false, true);     // dV, dK (A from TMEM)
+      constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);      // dQ = dS K
+      auto st_q = [&](int s) { return aSt + s * 2 * C::kTileBytes; };
+      auto st_do = [&](int s) { return aSt + s * 2 * C::kTileBytes + C::kTileBytes; };
+      // X^T = A B^T with both operands K-major: A = K or V (rows = keys), B = Q or dO.
+      auto kmajor_nt = [&](uint32_t dcol, uint32_t a, uint32_t bb) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_ss(tmem + dcol, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024), kIdS, k > 0);
+        }
+      };
+      // acc += X^T(tmem, packed bf16, 128 keys x 128 queries) * B(smem, queries x D, MN-major)
+      auto ts_acc = [&](uint32_t dcol, uint32_t acol, uint32_t bb, bool acc) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ts(tmem + dcol, tmem + acol + k * 8, sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&q_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        kmajor_nt(C::kColS, aK, st_q(0));
+        umma_commit(s_full);
+        kmajor_nt(C::kColDP, aV, st_do(0));
+        umma_commit(dp_full);
+      }
+      for (int it = 0; ok && it < total; ++it) {
+        const int s = it % C::kStages;
+        const int s1 = (it + 1) % C::kStages;
+        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
+        tc_fence_after();
+        ts_acc(C::kColDV, C::kColS, st_do(s), it > 0);  // dV += P^T dO
+        if (it + 1 < total) {
+          if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+          tc_fence_after();
+          kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
+          umma_commit(s_full);
+        }
+        if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
+        tc_fence_after();
+        ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
+        if (!C::kAliasDq && it > 0) {
+          if (!(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // dQ_i = dS K (both operands MN-major in smem)
+          umma_ss(tmem + C::kColDQ, sdesc_sw128(aDS + k * 2048, 16384, 1024),
+                  sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
+        umma_commit(dq_full);
+        umma_commit(&q_empty[s]);
+        if (it + 1 < total) {
+          if (C::kAliasDq) {
+            if (!(ok = mbar_wait(dq_empty, it & 1, abort_flag))) break;
+            tc_fence_after();
+          }
+          kmajor_nt(C::kColDP, aV, st_do(s1));  // dP^T of the next query tile
+          umma_commit(dp_full);
+        }
+      }
+      if (ok) umma_commit(kv_done);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P and dS (one key row per thread)
+    const int r = warp * 32 + lane;
+    const int key = k0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS;
+    const uint32_t tDP = tmem + lane_off + C::kColDP;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < total; ++it) {
+      const int i = q_tile(it);
+      const int q0 = i * 128;
+      const size_t vrow = static_cast<size_t>(q_head(it)) * p.Np + q0;
+      const float4* L4 = reinterpret_cast<const float4*>(p.lse2 + vrow);
+      const float4* D4 = reinterpret_cast<const float4*>(p.Drow + vrow);
+      bool full = true;  // every (query, key) pair of the tile allowed?
+      if (p.causal) full = full && (k0 + 127 <= q0);
+      if (p.window >= 0) full = full && (q0 + 127 - k0 <= p.window) && (k0 + 127 - q0 <= p.window);
+      if (!(ok = mbar_wait(s_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t pk[64];  // P^T row, packed bf16
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32];
+        tmem_ld32(tS + c * 32, sv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 l4 = __ldg(&L4[c * 8 + u]);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          float pv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int qc = c * 32 + u * 4 + e;
+            float x = fast_exp2(fmaf(__uint_as_float(sv[u * 4 + e]), sl2, -lv[e]));
+            if (!full) {
+              const int q = q0 + qc;
+              bool keep = true;
+              if (p.causal) keep = keep && key <= q;
+              if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
+              if (!keep) x = 0.f;
+            }
+            pv[e] = x;
+          }
+          pk[c * 16 + u * 2 + 0] = pack_bf16x2(pv[0], pv[1]);
+          pk[c * 16 + u * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+        }
+      }
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+
+      if (!(ok = mbar_wait(dp_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t dv[32];
+        tmem_ld32(tDP + c * 32, dv);
+        tmem_wait_ld();
+        uint32_t ds[16];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float4 d4 = __ldg(&D4[c * 8 + u]);
+          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&pk[c * 16 + u * 2 + e2]);
+            const float2 pf = __bfloat1622float2(pp);
+            const float g0 = pf.x * (__uint_as_float(dv[u * 4 + e2 * 2 + 0]) - dd[e2 * 2 + 0]);
+            const float g1 = pf.y * (__uint_as_float(dv[u * 4 + e2 * 2 + 1]) - dd[e2 * 2 + 1]);
+            ds[u * 2 + e2] = pack_bf16x2(g0, g1);
+          }
+        }
+        // dS^T (packed) into TMEM over dP^T columns already read; dS into shared
+        // memory as rows = keys, columns = queries (MN-major A operand of dQ).
+        tmem_st16(tDP + c * 16, ds);
+        const int chunk = c >> 1;
+        const int u0 = (c & 1) * 4;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 val = make_uint4(ds[4 * u], ds[4 * u + 1], ds[4 * u + 2], ds[4 * u + 3]);
+          *reinterpret_cast<uint4*>(sDS + chunk * 16384 + r * 128 + (((u0 + u) ^ (r & 7)) << 4)) = val;
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+  } else {
+    // ------------------------------------------------------------ dQ drain, then dK/dV epilogue
+    const int wl = warp & 3;
+    const int r = wl * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
+    bool ok = true;
+    for (int it = 0; it < total; ++it) {
+      if (!(ok = mbar_wait(dq_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t v[D];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c)
+        tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(dq_empty);
+      float* dst = p.dqacc + (static_cast<size_t>(q_head(it)) * p.Np + q_tile(it) * 128 + r) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 4) red_add_v4(dst + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+    }
+    if (ok) ok = mbar_wait(kv_done, 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      // K and V tiles are no longer read: stage dV over V and dK over K.
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + C::kColDV + c, v);
+        tmem_wait_ld();
+        stage_row32_bf16(sV, r, c, v, 1.f);
+        tmem_ld32(tmem + lane_off + C::kColDK + c, v);
+        tmem_wait_ld();
+        stage_row32_bf16(sK, r, c, v, p.scale);
+      }
+      fence_proxy_async_smem();
+    }
+    mbar_arrive(epi_bar);
+    if (ok && r == 0 && mbar_wait(epi_bar, 0, abort_flag)) {
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_store_3d(&tmdV, sV + c * 16384, c * 64, k0, bkv);
+        tma_store_3d(&tmdK, sK + c * 16384, c * 64, k0, bkv);
+      }
+      bulk_commit();
+      bulk_wait0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fa

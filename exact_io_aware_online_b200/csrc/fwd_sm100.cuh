@@ -1,0 +1,339 @@
+// fwd_sm100.cuh -- bf16 attention forward on sm_100a tensor cores.
+//
+// One CTA owns two 128-row query tiles of one (batch, head) and streams the
+// head's K/V tiles (128 keys each) through a TMA ring in shared memory.  For
+// every key tile it keeps, per query row, the online-softmax state of
+// "Flash attention and efficient attention" (section "Derivation: Incremental
+// Softmax"): the running maximum m, the running sum l and the unnormalised
+// accumulator O~, rescaled when the maximum moves (Step 3's merge with one new
+// block at a time).  Only O and the logsumexp reach global memory ("FlashAttention"
+// guide page, "Tiling through SRAM").
+//
+// Roles (320 threads):
+//   warps 0-3  softmax for query tile 0, one thread per row (TMEM lanes 0-127)
+//   warps 4-7  softmax for query tile 1
+//   warp 8     tcgen05.mma issuer (one thread) and TMEM owner
+//   warp 9     TMA producer (one thread)
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// P_t overwrites S_t as packed bf16 (64 columns) and is the A operand of the
+// P V product straight from TMEM, so P never touches shared memory.
+//
+// Differences from the pages' own design (which is SRAM tiling for an older
+// GPU): the scores live in TMEM, not registers or SRAM; exponentials are base 2
+// with the scale folded in; and the rescale of O~ is lazy -- the reference
+// maximum only moves when the new maximum exceeds it by more than kTau (log2
+// units), which keeps every p <= 2^kTau and is exact after the final 1/l.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  float* lse;
+  int B, H, Hkv, N, g;
+  float scale_log2;  // scale * log2(e)
+  int causal, window;
+  int npairs;     // ceil(N / 256): query-tile pairs per head
+  int ntiles_kv;  // ceil(N / 128)
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
+  static constexpr int kChunks = D / 64;          // 64-column (128-byte) chunks
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kSmemQ = 2 * kTileBytes;
+  static constexpr int kSmemKV = kStages * kTileBytes;
+  static constexpr int kNumBars = 1 + 2 * kStages + 8;
+  static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + 8 * kNumBars + 16;
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units (factor 256)
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                     const FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
+  uint8_t* sQ = base;
+  uint8_t* sKV = base + C::kSmemQ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + C::kSmemKV);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + C::kStages;
+  uint64_t* s_full = bars + 1 + 2 * C::kStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = s_full + 4;
+  uint64_t* epi_bar = s_full + 6;  // softmax threads -> storing thread: O tile staged
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work unit: heaviest (last) query-tile pairs first
+  const int BH = p.B * p.H;
+  const int pair = p.npairs - 1 - static_cast<int>(blockIdx.x) / BH;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.H, h = bh % p.H;
+  const int kvh = b * p.Hkv + h / p.g;
+  const int q0 = pair * 256;
+  const int qlast = min(q0 + 255, p.N - 1);
+  int jlo = 0, jhi = p.ntiles_kv - 1;
+  if (p.causal) jhi = min(jhi, qlast / 128);
+  if (p.window >= 0) {
+    jlo = max(0, q0 - p.window) / 128;
+    jhi = min(jhi, (qlast + p.window) / 128);
+  }
+  const int nkv = jhi - jlo + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+      mbar_init(&epi_bar[t], 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(&tmQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128, bh);
+      int issued[C::kStages];
+#pragma unroll
+      for (int i = 0; i < C::kStages; ++i) issued[i] = 0;
+      int it = 0;
+      for (int jj = 0; jj < nkv && !*abort_flag; ++jj) {
+        const int kv0 = (jlo + jj) * 128;
+        for (int which = 0; which < 2; ++which, ++it) {
+          const int s = it % C::kStages;
+          if (!mbar_wait(&kv_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
+          const CUtensorMap* m = which == 0 ? &tmK : &tmV;
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(m, &kv_full[s], sKV + s * C::kTileBytes + c * 16384, c * 64, kv0, kvh);
+          ++issued[s];
+        }
+      }
+      // Never leave the CTA with copies still landing in shared memory.
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(q_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
+      for (int s = 0; s < C::kStages; ++s)
+        if (issued[s] > 0)
+          while (!mbar_try_wait(smem_u32(&kv_full[s]), (issued[s] - 1) & 1) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV);
+      constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, false, true);
+      auto qk = [&](int t, int slot) {  // S_t = Q_t K^T
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
+          umma_ss(tmem + t * 128, sdesc_sw128(aQ + t * C::kTileBytes + off, 16, 1024),
+                  sdesc_sw128(aKV + slot * C::kTileBytes + off, 16, 1024), kIdescS, k > 0);
+        }
+      };
+      auto pv = [&](int t, int slot, bool acc) {  // O_t += P_t V
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8,
+                  sdesc_sw128(aKV + slot * C::kTileBytes + k * 2048, 16384, 1024), kIdescO, acc || k > 0);
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      int it = 0;
+      for (int jj = 0; ok && jj < nkv; ++jj, it += 2) {
+        const int sK = it % C::kStages;
+        if (!(ok = mbar_wait(&kv_full[sK], (it / C::kStages) & 1, abort_flag))) break;
+        tc_fence_after();
+        const int sVprev = (it - 1 + C::kStages) % C::kStages;
+        if (jj > 0) {
+          if (!(ok = mbar_wait(&p_full[0], (jj - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          pv(0, sVprev, jj > 1);
+        }
+        qk(0, sK);
+        umma_commit(&s_full[0]);
+        if (jj > 0) {
+          if (!(ok = mbar_wait(&p_full[1], (jj - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          pv(1, sVprev, jj > 1);
+          umma_commit(&kv_empty[sVprev]);
+        }
+        qk(1, sK);
+        umma_commit(&s_full[1]);
+        umma_commit(&kv_empty[sK]);
+        const int sV = (it + 1) % C::kStages;
+        if (!(ok = mbar_wait(&kv_full[sV], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+        tc_fence_after();
+      }
+      if (ok) {
+        const int sV = (it - 1) % C::kStages;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!(ok = mbar_wait(&p_full[t], (nkv - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          pv(t, sV, nkv > 1);
+          umma_commit(&o_full[t]);
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax (tile t)
+    const int t = warp >> 2;
+    const int wl = warp & 3;
+    const int r = wl * 32 + lane;
+    const int tq0 = q0 + t * 128;
+    const int qrow = tq0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * D;
+    const float sl2 = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int jj = 0; jj < nkv; ++jj) {
+      const int kv0 = (jlo + jj) * 128;
+      if (!(ok = mbar_wait(&s_full[t], jj & 1, abort_flag))) break;
+      tc_fence_after();
+      uint32_t sraw[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[c * 32]));
+      tmem_wait_ld();
+      float s[128];
+#pragma unroll
+      for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sraw[c]);
+      bool full = kv0 + 127 < p.N;
+      if (p.causal) full = full && (kv0 + 127 <= tq0);
+      if (p.window >= 0) full = full && (tq0 + 127 - kv0 <= p.window) && (kv0 + 127 - tq0 <= p.window);
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int key = kv0 + c;
+          bool keep = key < p.N;
+          if (p.causal) keep = keep && key <= qrow;
+          if (p.window >= 0) keep = keep && abs(qrow - key) <= p.window;
+          if (!keep) s[c] = -INFINITY;
+        }
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = fmaxf(m_used, mx * sl2);
+      bool need = false;
+      if (m_used == -INFINITY) {
+        m_used = m_new;  // nothing accumulated yet (or only exact zeros)
+      } else if (m_new > m_used + kTau) {
+        need = true;
+      }
+      if (__any_sync(0xffffffffu, need)) {
+        const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
+        if (need) {
+          l *= alpha;
+          m_used = m_new;
+        }
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + c, o);
+        }
+        tmem_wait_st();
+      }
+      const float ms = (m_used == -INFINITY) ? 0.f : m_used;
+      float rs = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = fast_exp2(fmaf(s[2 * c], sl2, -ms));
+        const float p1 = fast_exp2(fmaf(s[2 * c + 1], sl2, -ms));
+        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l += rs;
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+    if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      uint8_t* sO = sQ + t * C::kTileBytes;  // Q_t is no longer read
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c, o);
+        tmem_wait_ld();
+        const int chunk = c >> 6, u0 = (c & 63) >> 3;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          uint4 val;
+          val.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * inv, __uint_as_float(o[8 * u + 1]) * inv);
+          val.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv, __uint_as_float(o[8 * u + 3]) * inv);
+          val.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv, __uint_as_float(o[8 * u + 5]) * inv);
+          val.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
+          const uint32_t off = chunk * 16384 + r * 128 + (((u0 + u) ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(sO + off) = val;
+        }
+      }
+      if (qrow < p.N)
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      fence_proxy_async_smem();
+    }
+    // Every thread arrives (even after an abort) so the storing thread's
+    // bounded wait below cannot be left short of arrivals by a live peer.
+    mbar_arrive(&epi_bar[t]);
+    if (ok && r == 0 && tq0 < p.N && mbar_wait(&epi_bar[t], 0, abort_flag)) {
+      for (int c = 0; c < C::kChunks; ++c) tma_store_3d(&tmO, sQ + t * C::kTileBytes + c * 16384, c * 64, tq0, bh);
+      bulk_commit();
+      bulk_wait_read0();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace fa

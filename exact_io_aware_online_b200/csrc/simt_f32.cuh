@@ -1,0 +1,275 @@
+// simt_f32.cuh -- fp32 attention forward and backward on CUDA cores.
+//
+// The fp32 path keeps every product, exponential and sum in fp32 (tensor-core
+// TF32 would not meet a 1e-5 bound).  One warp owns one output row; its lanes
+// split the head dimension and reduce dot products with butterfly shuffles (all
+// lanes end with the identical sum, so the softmax state stays warp-uniform).
+// Key/value (or query/dO) rows are staged through shared memory, 32 at a time.
+//
+// Forward: online softmax over the allowed keys, one key at a time ("Flash
+// attention and efficient attention", "Derivation: Incremental Softmax": safe
+// softmax, and the Step 3 rescale whenever a new row maximum arrives).
+// Backward: S and P are recomputed from Q, K and the saved logsumexp ("Backward
+// Pass: Recomputation"); dQ is owned by query-row warps and dK/dV by key-row
+// warps, so nothing is accumulated with atomics and every result is
+// deterministic.
+#pragma once
+
+#include <stdint.h>
+
+namespace fa {
+
+struct SimtParams {
+  const float* q;
+  const float* k;
+  const float* v;
+  const float* o;
+  const float* dout;
+  const float* lse;
+  float* o_out;
+  float* lse_out;
+  float* dq;
+  float* dk;
+  float* dv;
+  float* Drow;  // workspace: D_i = sum_k dO_ik O_ik, [B*H*N]
+  int B, H, Hkv, N, g;
+  float scale;
+  int causal, window;
+};
+
+__device__ __forceinline__ bool keep_ij(int i, int j, int causal, int window) {
+  return (!causal || j <= i) && (window < 0 || abs(i - j) <= window);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+constexpr int kSimtRows = 8;  // warps (rows) per block
+constexpr int kSimtTile = 32;  // staged rows per smem tile
+
+// Keys that query rows [r0, r1) may see: [lo, hi).
+__device__ __forceinline__ void simt_key_range(int r0, int r1, int N, int causal, int window, int& lo, int& hi) {
+  lo = 0;
+  hi = N;
+  if (causal) hi = min(hi, r1);
+  if (window >= 0) {
+    lo = max(lo, r0 - window);
+    hi = min(hi, r1 + window);
+  }
+}
+// Query rows that keys [c0, c1) are seen by: [lo, hi).
+__device__ __forceinline__ void simt_query_range(int c0, int c1, int N, int causal, int window, int& lo, int& hi) {
+  lo = 0;
+  hi = N;
+  if (causal) lo = max(lo, c0);
+  if (window >= 0) {
+    lo = max(lo, c0 - window);
+    hi = min(hi, c1 + window);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
+  constexpr int E = D / 32;
+  __shared__ float sK[kSimtTile][D];
+  __shared__ float sV[kSimtTile][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+  const int kvh = b * p.Hkv + h / p.g;
+  const int r0 = blockIdx.x * kSimtRows, r1 = min(p.N, r0 + kSimtRows);
+  const int i = r0 + warp;
+  const bool active = i < p.N;
+  const float* qrow = p.q + (static_cast<size_t>(bh) * p.N + (active ? i : 0)) * D;
+  const float* kbase = p.k + static_cast<size_t>(kvh) * p.N * D;
+  const float* vbase = p.v + static_cast<size_t>(kvh) * p.N * D;
+  float q[E], acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    q[e] = qrow[lane + 32 * e];
+    acc[e] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  int lo, hi;
+  simt_key_range(r0, r1, p.N, p.causal, p.window, lo, hi);
+  for (int kt = lo; kt < hi; kt += kSimtTile) {
+    const int cnt = min(kSimtTile, hi - kt);
+    __syncthreads();
+    for (int x = threadIdx.x; x < cnt * D; x += blockDim.x) {
+      sK[x / D][x % D] = kbase[static_cast<size_t>(kt) * D + x];
+      sV[x / D][x % D] = vbase[static_cast<size_t>(kt) * D + x];
+    }
+    __syncthreads();
+    if (!active) continue;
+    for (int jj = 0; jj < cnt; ++jj) {
+      const int j = kt + jj;
+      if (!keep_ij(i, j, p.causal, p.window)) continue;
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) s = fmaf(q[e], sK[jj][lane + 32 * e], s);
+      s = warp_sum(s) * p.scale;
+      if (s > m) {  // a new row maximum: rescale what was accumulated
+        const float a = expf(m - s);
+        l *= a;
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] *= a;
+        m = s;
+      }
+      const float pe = expf(s - m);
+      l += pe;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, sV[jj][lane + 32 * e], acc[e]);
+    }
+  }
+  if (!active) return;
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  float* orow = p.o_out + (static_cast<size_t>(bh) * p.N + i) * D;
+#pragma unroll
+  for (int e = 0; e < E; ++e) orow[lane + 32 * e] = acc[e] * inv;
+  if (lane == 0) p.lse_out[static_cast<size_t>(bh) * p.N + i] = l > 0.f ? m + logf(l) : -INFINITY;
+}
+
+// D_i = sum_k dO_ik O_ik (equal to sum_j P_ij dP_ij, the softmax-Jacobian row term).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_rowdot_f32_kernel(const SimtParams p) {
+  constexpr int E = D / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t row = static_cast<size_t>(blockIdx.x) * kSimtRows + warp;
+  if (row >= static_cast<size_t>(p.B) * p.H * p.N) return;
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) s = fmaf(p.dout[row * D + lane + 32 * e], p.o[row * D + lane + 32 * e], s);
+  s = warp_sum(s);
+  if (lane == 0) p.Drow[row] = s;
+}
+
+// dK, dV: one warp per key row of a kv head, summing over its query heads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
+  constexpr int E = D / 32;
+  __shared__ float sQ[kSimtTile][D];
+  __shared__ float sO[kSimtTile][D];  // dO rows
+  __shared__ float sL[kSimtTile], sD[kSimtTile];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bkv = blockIdx.y, b = bkv / p.Hkv, kh = bkv % p.Hkv;
+  const int c0 = blockIdx.x * kSimtRows, c1 = min(p.N, c0 + kSimtRows);
+  const int j = c0 + warp;
+  const bool active = j < p.N;
+  const float* krow = p.k + (static_cast<size_t>(bkv) * p.N + (active ? j : 0)) * D;
+  const float* vrow = p.v + (static_cast<size_t>(bkv) * p.N + (active ? j : 0)) * D;
+  float kk[E], vv[E], dk[E], dv[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    kk[e] = krow[lane + 32 * e];
+    vv[e] = vrow[lane + 32 * e];
+    dk[e] = 0.f;
+    dv[e] = 0.f;
+  }
+  int lo, hi;
+  simt_query_range(c0, c1, p.N, p.causal, p.window, lo, hi);
+  for (int hq = 0; hq < p.g; ++hq) {
+    const int bh = b * p.H + kh * p.g + hq;
+    const float* qbase = p.q + static_cast<size_t>(bh) * p.N * D;
+    const float* obase = p.dout + static_cast<size_t>(bh) * p.N * D;
+    for (int it = lo; it < hi; it += kSimtTile) {
+      const int cnt = min(kSimtTile, hi - it);
+      __syncthreads();
+      for (int x = threadIdx.x; x < cnt * D; x += blockDim.x) {
+        sQ[x / D][x % D] = qbase[static_cast<size_t>(it) * D + x];
+        sO[x / D][x % D] = obase[static_cast<size_t>(it) * D + x];
+      }
+      for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
+        sL[x] = p.lse[static_cast<size_t>(bh) * p.N + it + x];
+        sD[x] = p.Drow[static_cast<size_t>(bh) * p.N + it + x];
+      }
+      __syncthreads();
+      if (!active) continue;
+      for (int ii = 0; ii < cnt; ++ii) {
+        const int i = it + ii;
+        if (!keep_ij(i, j, p.causal, p.window)) continue;
+        float s = 0.f, dp = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          s = fmaf(sQ[ii][lane + 32 * e], kk[e], s);
+          dp = fmaf(sO[ii][lane + 32 * e], vv[e], dp);
+        }
+        s = warp_sum(s) * p.scale;
+        dp = warp_sum(dp);
+        const float pr = expf(s - sL[ii]);
+        const float ds = pr * (dp - sD[ii]);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          dv[e] = fmaf(pr, sO[ii][lane + 32 * e], dv[e]);
+          dk[e] = fmaf(ds, sQ[ii][lane + 32 * e], dk[e]);
+        }
+      }
+    }
+  }
+  if (!active) return;
+  float* dkrow = p.dk + (static_cast<size_t>(bkv) * p.N + j) * D;
+  float* dvrow = p.dv + (static_cast<size_t>(bkv) * p.N + j) * D;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    dkrow[lane + 32 * e] = dk[e] * p.scale;
+    dvrow[lane + 32 * e] = dv[e];
+  }
+}
+
+// dQ: one warp per query row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_f32_kernel(const SimtParams p) {
+  constexpr int E = D / 32;
+  __shared__ float sK[kSimtTile][D];
+  __shared__ float sV[kSimtTile][D];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+  const int kvh = b * p.Hkv + h / p.g;
+  const int r0 = blockIdx.x * kSimtRows, r1 = min(p.N, r0 + kSimtRows);
+  const int i = r0 + warp;
+  const bool active = i < p.N;
+  const size_t row = static_cast<size_t>(bh) * p.N + (active ? i : 0);
+  float q[E], dO[E], dq[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    q[e] = p.q[row * D + lane + 32 * e];
+    dO[e] = p.dout[row * D + lane + 32 * e];
+    dq[e] = 0.f;
+  }
+  const float L = p.lse[row], Dr = p.Drow[row];
+  const float* kbase = p.k + static_cast<size_t>(kvh) * p.N * D;
+  const float* vbase = p.v + static_cast<size_t>(kvh) * p.N * D;
+  int lo, hi;
+  simt_key_range(r0, r1, p.N, p.causal, p.window, lo, hi);
+  for (int kt = lo; kt < hi; kt += kSimtTile) {
+    const int cnt = min(kSimtTile, hi - kt);
+    __syncthreads();
+    for (int x = threadIdx.x; x < cnt * D; x += blockDim.x) {
+      sK[x / D][x % D] = kbase[static_cast<size_t>(kt) * D + x];
+      sV[x / D][x % D] = vbase[static_cast<size_t>(kt) * D + x];
+    }
+    __syncthreads();
+    if (!active) continue;
+    for (int jj = 0; jj < cnt; ++jj) {
+      const int j = kt + jj;
+      if (!keep_ij(i, j, p.causal, p.window)) continue;
+      float s = 0.f, dp = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        s = fmaf(q[e], sK[jj][lane + 32 * e], s);
+        dp = fmaf(dO[e], sV[jj][lane + 32 * e], dp);
+      }
+      s = warp_sum(s) * p.scale;
+      dp = warp_sum(dp);
+      const float ds = expf(s - L) * (dp - Dr);
+#pragma unroll
+      for (int e = 0; e < E; ++e) dq[e] = fmaf(ds, sK[jj][lane + 32 * e], dq[e]);
+    }
+  }
+  if (!active) return;
+#pragma unroll
+  for (int e = 0; e < E; ++e) p.dq[row * D + lane + 32 * e] = dq[e] * p.scale;
+}
+
+}  // namespace fa

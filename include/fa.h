@@ -1,0 +1,115 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact softmax attention, forward and backward,
+ * computed tile by tile with the online-softmax state on NVIDIA B200 (sm_100a).
+ *
+ * What is computed (per batch b and query head h, kv head kh = h / (H / Hkv)):
+ *   S = scale * Q K^T, masked;  P = softmax(S) row-wise;  O = P V
+ * ("Flash attention and efficient attention", section "The Standard Attention
+ * Problem"; the scale there is 1/sqrt(d_k) and is an argument here).  The N x N
+ * matrices S and P are never written to device memory: only O and the per-row
+ * logsumexp LSE are ("FlashAttention" guide page, section "Tiling through
+ * SRAM").  The backward recomputes S and P per tile from Q, K, V and LSE
+ * ("Flash attention and efficient attention", section "Backward Pass:
+ * Recomputation") and returns the gradients of L = sum(dO * O).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Layouts   all tensors contiguous, row-major, head dim d fastest:
+ *              q, o, dout, dq      [B, H,   N, d]
+ *              k, v, dk, dv        [B, Hkv, N, d]
+ *              lse                 [B, H,   N]   fp32, natural log of
+ *                                  sum_j exp(S_ij) over the allowed keys
+ *  dtype     FA_BF16: q/k/v/o/dout/dq/dk/dv are bfloat16 (fp32 accumulation);
+ *            FA_FP32: they are float.  lse and the workspace are always float.
+ *  Masks     causal != 0 keeps keys j <= i; window >= 0 keeps |i - j| <= window
+ *            (half-width: the pages' "w = 3, itself plus one neighbour each
+ *            side" is window = 1); window = -1 disables the band; both may be
+ *            combined (i - window <= j <= i).
+ *  Sizes     B, H, Hkv, N >= 1; H % Hkv == 0; d in {64, 128};
+ *            scale finite and > 0.
+ *  Pointers  device pointers (cudaMalloc'd or equivalent), 16-byte aligned;
+ *            outputs must not alias inputs (not checked).  The caller owns all
+ *            memory; the library allocates no device memory.
+ *  stream    a cudaStream_t passed as void*; NULL means the legacy default
+ *            stream.  Every call only enqueues work and returns without
+ *            synchronising; results are ready when the stream reaches them.
+ *  Errors    argument errors are detected on the host before anything is
+ *            enqueued and leave all buffers untouched; a failed launch returns
+ *            FA_ERR_CUDA.  A device-side bounded wait that gives up (after about
+ *            two seconds) records FA_ERR_TIMEOUT in a device status word that
+ *            fa_last_device_status() reports.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, size < 1, H % Hkv != 0, bad scale/window/dtype */
+  FA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. d not in {64, 128}) */
+  FA_ERR_MISALIGNED = 3,  /* a pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = 4,   /* workspace pointer null or ws_bytes too small */
+  FA_ERR_CUDA = 5,        /* a CUDA runtime/driver call or a launch failed */
+  FA_ERR_TIMEOUT = 6      /* a device-side bounded wait gave up */
+} fa_status;
+
+typedef enum fa_dtype { FA_BF16 = 0, FA_FP32 = 1 } fa_dtype;
+
+/*
+ * Forward: o = softmax(scale * q k^T, masked) v and lse (see above).
+ * The online-softmax recurrence (running max m, running sum l, rescaled
+ * unnormalised accumulator) is the one of "Flash attention and efficient
+ * attention", section "Derivation: Incremental Softmax", Steps 1-3, applied
+ * block after block of keys ("This generalizes to any number of blocks").
+ * Writes o [B,H,N,d] and lse [B,H,N]; reads q, k, v.  Deterministic.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int Hkv, int N, int d, float scale, int causal, int window,
+                 fa_dtype dtype, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs for these sizes (fp32 row terms
+ * D_i = sum_k dO_ik O_ik, prescaled LSE, and for bf16 a float dQ accumulator).
+ * Returns 0 for sizes fa_bwd would reject.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype);
+
+/*
+ * Backward of fa_fwd for the loss L = sum(dout * o): writes dq [B,H,N,d],
+ * dk and dv [B,Hkv,N,d].  Reads q, k, v, o, dout and the lse that fa_fwd wrote
+ * for the same inputs; recomputes S and P per tile ("Flash attention and
+ * efficient attention", "Backward Pass: Recomputation").  The gradients of a
+ * kv head sum over its H / Hkv query heads.  workspace: caller-owned device
+ * memory of at least fa_bwd_workspace_size() bytes, 16-byte aligned; its
+ * contents on entry do not matter and are garbage on return.  dk, dv, o and
+ * lse are deterministic; dq (bf16 path) sums tile contributions with atomics,
+ * so its last bits may vary from run to run.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                 int B, int H, int Hkv, int N, int d, float scale, int causal, int window,
+                 fa_dtype dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word:
+ * FA_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call,
+ * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK.
+ */
+fa_status fa_last_device_status(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fa_status_string(fa_status s);
+
+/* Library ABI version (major * 100 + minor). */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,105 @@
+"""C-ABI boundary checks that need no GPU: the library loads, exports every
+symbol the header declares, and rejects bad arguments on the host before
+touching the device (so fake, never-dereferenced pointer values are safe)."""
+import ctypes
+import subprocess
+
+import pytest
+
+import exact_io_aware_online_b200 as fa
+from exact_io_aware_online_b200 import _build
+
+A = 0x7f0000010000  # a 16-byte aligned fake device address (never dereferenced on these paths)
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return fa.lib()
+
+
+def test_header_declares_expected_entry_points():
+    names = fa.exported_names()
+    for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
+              "fa_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in fa.exported_names():
+        assert n in exported, n
+        assert getattr(L, n) is not None
+
+
+def test_status_strings_and_version(L):
+    assert L.fa_version() == 100
+    for code in range(7):
+        assert L.fa_status_string(code)
+    assert L.fa_status_string(99) == b"unknown status"
+
+
+def _fwd(L, **kw):
+    a = dict(q=A, k=A, v=A, o=A, lse=A, B=1, H=2, Hkv=1, N=16, d=64, scale=0.125, causal=0, window=-1, dtype=0)
+    a.update(kw)
+    return L.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Hkv"], a["N"], a["d"],
+                    ctypes.c_float(a["scale"]), a["causal"], a["window"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(o=None), 1), (dict(lse=None), 1),
+    (dict(B=0), 1), (dict(H=0), 1), (dict(Hkv=0), 1), (dict(N=0), 1), (dict(N=-5), 1),
+    (dict(H=3, Hkv=2), 1), (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1),
+    (dict(scale=float("inf")), 1), (dict(window=-2), 1), (dict(dtype=7), 1),
+    (dict(d=32), 2), (dict(d=96), 2), (dict(d=256), 2),
+    (dict(q=A + 8), 3), (dict(k=A + 4), 3), (dict(o=A + 2), 3), (dict(lse=A + 12), 3),
+])
+def test_fwd_rejects_bad_arguments(L, kw, code):
+    assert _fwd(L, **kw) == code
+
+
+def _bwd(L, ws=A, ws_bytes=None, **kw):
+    a = dict(B=1, H=2, Hkv=1, N=16, d=64, scale=0.125, causal=0, window=-1, dtype=0)
+    a.update(kw)
+    if ws_bytes is None:
+        ws_bytes = L.fa_bwd_workspace_size(a["B"], a["H"], a["N"], a["d"], a["dtype"] if a["dtype"] in (0, 1) else 0)
+    ptrs = [kw.get(n, A) for n in ("q", "k", "v", "o", "do", "lse", "dq", "dk", "dv")]
+    return L.fa_bwd(*ptrs, ws, ws_bytes, a["B"], a["H"], a["Hkv"], a["N"], a["d"], ctypes.c_float(a["scale"]),
+                    a["causal"], a["window"], a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(do=None), 1), (dict(lse=None), 1), (dict(dq=None), 1), (dict(dv=None), 1),
+    (dict(H=4, Hkv=3), 1), (dict(window=-3), 1), (dict(scale=0.0), 1), (dict(d=80), 2),
+    (dict(dk=A + 8), 3), (dict(do=A + 4), 3),
+    (dict(ws=None), 4), (dict(ws_bytes=16), 4), (dict(ws=A + 8), 3),
+])
+def test_bwd_rejects_bad_arguments(L, kw, code):
+    assert _bwd(L, **kw) == code
+
+
+def test_bwd_workspace_one_byte_short_is_rejected(L):
+    need = L.fa_bwd_workspace_size(2, 4, 300, 128, 0)
+    assert _bwd(L, ws_bytes=need - 1, B=2, H=4, Hkv=2, N=300, d=128) == 4
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 1, 1, 64), (2, 16, 8192, 128), (1, 32, 16384, 128), (3, 5, 130, 64)])
+def test_workspace_size_closed_form(L, B, H, N, d):
+    def a256(x):
+        return (x + 255) // 256 * 256
+    np_ = (N + 127) // 128 * 128
+    rows = B * H * np_
+    assert L.fa_bwd_workspace_size(B, H, N, d, 0) == a256(rows * 4) * 2 + a256(rows * d * 4)
+    assert L.fa_bwd_workspace_size(B, H, N, d, 1) == a256(B * H * N * 4)
+    assert L.fa_bwd_workspace_size(B, H, N, 96, 0) == 0
+    assert L.fa_bwd_workspace_size(0, H, N, d, 0) == 0
+
+
+def test_python_helpers_fail_loudly_without_cuda():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(Exception):
+        fa.fwd(q, q, q)

@@ -1,0 +1,126 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU fp64 oracle on
+the same seeded inputs.
+
+Small cases cover every output element and span several tiles plus a ragged
+tail; the full-size workloads run in the launch configuration the benchmark
+times and are compared on whole sampled heads (whole GQA groups).
+"""
+import pytest
+import torch
+
+import exact_io_aware_online_b200 as fa
+from exact_io_aware_online_b200 import workloads as W
+
+from parity_util import check_groups, gpu_run, oracle_groups
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from exact_io_aware_online_b200 import _build
+    _build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+
+
+def _case(name, B, H, Hkv, N, d, dtype, causal, window, seed=11, boost=0.0):
+    return W.Workload(name, B, H, Hkv, N, d, dtype, causal, window, seed, boost)
+
+
+def _all_groups(w):
+    return [(b, kh) for b in range(w.B) for kh in range(w.Hkv)]
+
+
+SMALL = [
+    # name, B, H, Hkv, N, d, dtype, causal, window
+    ("n1_d64", 1, 1, 1, 1, 64, False, -1),
+    ("n17_causal_d64", 1, 2, 1, 17, 64, True, -1),
+    ("n128_d128", 2, 2, 2, 128, 128, False, -1),
+    ("n130_causal_d128", 1, 2, 1, 130, 128, True, -1),
+    ("n383_causal_gqa_d64", 1, 4, 2, 383, 64, True, -1),
+    ("n512_window5_d128", 1, 2, 2, 512, 128, False, 5),
+    ("n700_window128_d64", 1, 2, 2, 700, 64, False, 128),
+    ("n300_causal_window64_d128", 1, 2, 1, 300, 128, True, 64),
+    ("n1024_causal_d128", 1, 1, 1, 1024, 128, True, -1),
+    ("n256_gqa4_d64", 2, 4, 1, 256, 64, False, -1),
+    ("n640_window0_d64", 1, 1, 1, 640, 64, False, 0),
+    ("n900_boost_causal_gqa_d128", 1, 4, 2, 900, 128, True, -1),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_small_cases_every_element(case, dtype):
+    name, B, H, Hkv, N, d, causal, window = case
+    w = _case(name, B, H, Hkv, N, d, dtype, causal, window, boost=0.05 if "boost" in name else 0.0)
+    x = W.make_inputs(w)
+    got = gpu_run(w, x)
+    want = oracle_groups(w, x, _all_groups(w))
+    check_groups(w, got, want)
+
+
+def test_fp32_workload_every_element():
+    w = W.WORKLOADS["fp32_n256_d64"]
+    x = W.make_inputs(w)
+    got = gpu_run(w, x)
+    want = oracle_groups(w, x, _all_groups(w))
+    check_groups(w, got, want)
+
+
+FULL = {
+    "bf16_b4h16_n2048_d64": [(0, 0), (3, 15)],
+    "bf16_causal_b2h16_n8192_d128": [(0, 0), (1, 9)],
+    "bf16_gqa_causal_h32kv8_n16384_d128": [(0, 5)],
+    "bf16_window128_h16_n32768_d64": [(0, 0), (0, 13)],
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_workload_sampled_heads(name):
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w)
+    got = gpu_run(w, x)
+    want = oracle_groups(w, x, FULL[name])
+    worst = check_groups(w, got, want)
+    print(name, worst)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_deterministic_outputs(dtype):
+    w = _case("det", 1, 4, 2, 777, 128, dtype, True, -1)
+    x = {k: t.cuda() for k, t in W.make_inputs(w).items()}
+    o1, l1 = fa.fwd(x["q"], x["k"], x["v"], w.scale, True)
+    o2, l2 = fa.fwd(x["q"], x["k"], x["v"], w.scale, True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    g1 = fa.bwd(x["q"], x["k"], x["v"], o1, l1, x["do"], w.scale, True)
+    g2 = fa.bwd(x["q"], x["k"], x["v"], o1, l1, x["do"], w.scale, True)
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+    assert torch.allclose(g1[0].float(), g2[0].float(), rtol=0, atol=1e-2)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_nothing_written_outside_outputs(dtype):
+    """Outputs live inside larger buffers filled with a sentinel; only the
+    output ranges may change."""
+    w = _case("canary", 1, 2, 1, 300, 64, dtype, True, -1)
+    x = {k: t.cuda() for k, t in W.make_inputs(w).items()}
+    dt = x["q"].dtype
+    pad = 4096
+
+    def guarded(shape, dtype_):
+        n = 1
+        for s in shape:
+            n *= s
+        buf = torch.full((n + 2 * pad,), -7777.0, dtype=dtype_, device="cuda")
+        return buf, buf[pad:pad + n].view(shape)
+
+    ob, o = guarded(x["q"].shape, dt)
+    lb, lse = guarded(x["q"].shape[:3], torch.float32)
+    fa.fwd(x["q"], x["k"], x["v"], w.scale, True, out=o, lse=lse)
+    bufs = [guarded(x["q"].shape, dt), guarded(x["k"].shape, dt), guarded(x["v"].shape, dt)]
+    fa.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], w.scale, True, grads=tuple(b[1] for b in bufs))
+    torch.cuda.synchronize()
+    for buf, _ in [(ob, o), (lb, lse)] + bufs:
+        assert (buf[:pad] == -7777.0).all() and (buf[-pad:] == -7777.0).all()
+    assert fa.device_status() == 0
