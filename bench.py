@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward + backward on B200 through the C ABI.
+
+One step = fa_fwd + fa_bwd over the whole workload (default: the causal
+bf16 B=2 H=16 N=8192 d=128 workload), inputs already resident in device memory.
+Prints one JSON line (rank 0).  Throughput counts 4*N^2*d flops per head
+forward and 2.5x that backward, halved for causal.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+copy of the workload (a different seed), with no data-path collective; the
+timed region is bracketed by barriers and the reported time is the maximum
+over ranks ("weak" scaling).  --impl reference times the CPU fp64 oracle (the
+only other implementation of this path) on a bounded sample of the workload,
+on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_online_b200 import workloads as W  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_online_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if it
+    was captured on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}@{workload}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.rows = []
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) == 9:
+                self.rows.append(parts)
+
+    def summary(self):
+        if not getattr(self, "rows", None):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        mhz = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in self.rows if r[2].replace(".", "").isdigit()]
+        power = [float(r[3]) for r in self.rows if r[3].replace(".", "").isdigit()]
+        load = [m for m in mhz] or [0.0]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows), "power_w_max": max(power) if power else None}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        if args.impl == "ours":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=600))
+    return world, rank, local
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_sample(w: W.Workload, min_seconds: float, max_heads: int):
+    """Times the CPU oracle (fwd + bwd) on whole query heads of the workload until
+    at least `min_seconds` have elapsed.  Returns (seconds, flops, heads)."""
+    from oracle import ref
+    x = W.make_inputs(w)
+    g = w.H // w.Hkv
+    fwd_f, bwd_f = W.flops(w)
+    per_head = (fwd_f + bwd_f) / (w.B * w.H)
+    spent, heads = 0.0, 0
+    order = [(b, h) for h in range(w.H) for b in range(w.B)]
+    for b, h in order[:max_heads]:
+        kh = h // g
+        q, do = x["q"][b:b + 1, h:h + 1], x["do"][b:b + 1, h:h + 1]
+        k, v = x["k"][b:b + 1, kh:kh + 1], x["v"][b:b + 1, kh:kh + 1]
+        t0 = time.perf_counter()
+        ref.forward(q, k, v, w.scale, w.causal, w.window)
+        ref.backward(q, k, v, do, w.scale, w.causal, w.window)
+        spent += time.perf_counter() - t0
+        heads += 1
+        if spent >= min_seconds:
+            break
+    return spent, per_head * heads, heads
+
+
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return 0
+    fwd_f, bwd_f = W.flops(w)
+    per_head = (fwd_f + bwd_f) / (w.B * w.H)
+    from oracle import ref
+    x = W.make_inputs(w)
+    g = w.H // w.Hkv
+    q, do = x["q"][0:1, 0:1], x["do"][0:1, 0:1]
+    k, v = x["k"][0:1, 0:1], x["v"][0:1, 0:1]
+
+    def step():
+        ref.forward(q, k, v, w.scale, w.causal, w.window)
+        ref.backward(q, k, v, do, w.scale, w.causal, w.window)
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = per_head / sec / 1e12
+    sample = f"one query head (b=0, h=0; kv head 0) of {w.name}, forward+backward, every row"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "attention fwd+bwd TFLOP/s (bf16, causal N=8192 d=128) and % of BF16 tensor peak"
+
+
+def config_of(w: W.Workload, world: int):
+    in_bytes = (2 * w.B * w.H + 2 * w.B * w.Hkv) * w.N * w.d * (2 if w.dtype == "bf16" else 4)
+    return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+            "window": w.window, "scale": "1/sqrt(d)", "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of Q,K,V,dO per step per GPU (no flush)"}
+
+
+def run_ours(args, w, world, rank, local):
+    import torch
+    import exact_io_aware_online_b200 as fa
+    from exact_io_aware_online_b200 import _build
+
+    if rank == 0:
+        _build.build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.lib()
+    wr = w.with_(seed=w.seed + 1000 * rank)
+    host = W.make_inputs(wr)
+    x = {k: t.to(dev) for k, t in host.items()}
+    B, H, N, d = x["q"].shape
+    o = torch.empty_like(x["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d, fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP32),
+                     dtype=torch.uint8, device=dev)
+    K = args.steps
+    ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+    def step(i=None):
+        if i is not None:
+            fa.set_timing_events(*ev_f[i])
+        fa.fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, out=o, lse=lse)
+        if i is not None:
+            fa.set_timing_events(*ev_b[i])
+        fa.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], w.scale, w.causal, w.window, workspace=ws,
+               grads=(dq, dk, dv))
+        if i is not None:
+            fa.set_timing_events(None, None)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.device_status() != 0:
+        raise RuntimeError("device-side timeout during warm-up")
+    stream = torch.cuda.current_stream(dev)
+    t_start, t_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_start.record(stream)
+        for i in range(K):
+            step(i)
+        t_stop.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    if fa.device_status() != 0:
+        raise RuntimeError("device-side timeout during the timed region")
+    ms = t_start.elapsed_time(t_stop)
+    fwd_ms = [a.elapsed_time(b) for a, b in ev_f]
+    bwd_ms = [a.elapsed_time(b) for a, b in ev_b]
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    fwd_f, bwd_f = W.flops(w)
+    ms_step = ms / K
+    value = world * (fwd_f + bwd_f) / (ms_step * 1e-3) / 1e12
+
+    pk, src = peaks()
+    fwd_k, bwd_k = statistics.mean(fwd_ms), statistics.mean(bwd_ms)
+    if bwd_k * bwd_f >= 0 and bwd_k >= fwd_k:
+        dom_name, dom_ms, dom_flops = "bwd_sm100_kernel", bwd_k, bwd_f
+    else:
+        dom_name, dom_ms, dom_flops = "fwd_sm100_kernel", fwd_k, fwd_f
+    if w.dtype != "bf16":
+        dom_name = dom_name.replace("sm100", "simt_f32")
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = float(pk["bf16_tflops_sustained"])
+    roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": ncu_traffic(dom_name, w.name),
+            "peak_kind": f"bf16 dense, sustained ({src})",
+            "frac_of_burst_peak": achieved / float(pk["bf16_tflops"]),
+            "fwd_kernel_ms": fwd_k, "bwd_kernel_ms": bwd_k,
+            "fwd_kernel_tflops": fwd_f / (fwd_k * 1e-3) / 1e12,
+            "bwd_kernel_tflops": bwd_f / (bwd_k * 1e-3) / 1e12}
+
+    # ---- end to end: pinned host inputs -> device, fwd+bwd, results -> pinned host
+    e2e = None
+    if not args.no_e2e:
+        hin = {k: t.pin_memory() for k, t in host.items()}
+        hout = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+                "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory(),
+                "dq": torch.empty(dq.shape, dtype=dq.dtype).pin_memory(),
+                "dk": torch.empty(dk.shape, dtype=dk.dtype).pin_memory(),
+                "dv": torch.empty(dv.shape, dtype=dv.dtype).pin_memory()}
+
+        def e2e_step():
+            for k_ in ("q", "k", "v", "do"):
+                x[k_].copy_(hin[k_], non_blocking=True)
+            step()
+            for k_, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+                hout[k_].copy_(t, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = a.elapsed_time(b_)
+        if world > 1:
+            import torch.distributed as dist
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = sum(t.numel() * t.element_size() for t in hin.values())
+        d2h = sum(t.numel() * t.element_size() for t in hout.values())
+        e2e = {"value": world * (fwd_f + bwd_f) / (ems / K * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ems / K}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sec, flops_done, heads = oracle_sample(w, args.cpu_seconds, w.B * w.H)
+        cpu = {"value": flops_done / sec / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"{heads} whole query head(s) of {w.name} (fwd+bwd, every row), {sec:.1f} s",
+               "host_cpus": os.cpu_count()}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": config_of(w, world), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "clocks": clk.summary(), "gpu_launches": K * (1 + 3),
+            "frac_of_peak": {"sustained": value / world / float(pk["bf16_tflops_sustained"]),
+                             "burst": value / world / float(pk["bf16_tflops"]), "peaks": src},
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=W.HEADLINE, choices=list(W.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    w = W.WORKLOADS[args.workload]
+    try:
+        if args.impl == "reference":
+            return run_reference(args, w, world, rank)
+        return run_ours(args, w, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -14,7 +14,7 @@ import os
 import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
-           "exported_names", "LIB_PATH", "HEADER_PATH"]
+           "exported_names", "set_timing_events", "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_version.argtypes = []
     L.fa_version.restype = i
+    L.fa_set_timing_events.argtypes = [vp, vp]
+    L.fa_set_timing_events.restype = None
     _lib = L
     return L
 
@@ -122,6 +124,12 @@ def bwd(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, w
                         _stream_ptr(q.device))
     _check(code, "fa_bwd")
     return dq, dk, dv
+
+
+def set_timing_events(start=None, stop=None):
+    """Record torch.cuda.Event pair around the next calls' main kernel (None: off)."""
+    lib().fa_set_timing_events(start.cuda_event if start is not None else None,
+                               stop.cuda_event if stop is not None else None)
 
 
 def device_status(device=None) -> int:

@@ -17,6 +17,14 @@ namespace {
 
 constexpr int kAbiVersion = 100;
 
+cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;  // fa_set_timing_events
+inline void mark_start(cudaStream_t st) {
+  if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_start, st);
+}
+inline void mark_stop(cudaStream_t st) {
+  if (g_ev_start && g_ev_stop) cudaEventRecord(g_ev_stop, st);
+}
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 fa_status check_common(int B, int H, int Hkv, int N, int d, float scale, int window, fa_dtype dtype) {
@@ -111,7 +119,9 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   p.npairs = (N + 255) / 256;
   p.ntiles_kv = (N + 127) / 128;
   const unsigned grid = static_cast<unsigned>(p.npairs) * B * H;
+  mark_start(st);
   fa::fwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+  mark_stop(st);
   return launched();
 }
 
@@ -125,7 +135,9 @@ fa_status fwd_f32(const void* q, const void* k, const void* v, void* o, float* l
   s.o_out = static_cast<float*>(o);
   s.lse_out = lse;
   dim3 grid((N + fa::kSimtRows - 1) / fa::kSimtRows, B * H);
+  mark_start(st);
   fa::fwd_simt_f32_kernel<D><<<grid, 32 * fa::kSimtRows, 0, st>>>(s);
+  mark_stop(st);
   return launched();
 }
 
@@ -183,7 +195,9 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   fa::bwd_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.ntiles) * B * Hkv;
+  mark_start(st);
   fa::bwd_sm100_kernel<D><<<grid, 320, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
+  mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   const size_t n4 = static_cast<size_t>(B) * H * N * D / 4;
   fa::bwd_dq_kernel<D><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p);
@@ -210,7 +224,9 @@ fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, co
                                  32 * fa::kSimtRows, 0, st>>>(s);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   dim3 gkv((N + fa::kSimtRows - 1) / fa::kSimtRows, B * Hkv);
+  mark_start(st);
   fa::bwd_dkdv_f32_kernel<D><<<gkv, 32 * fa::kSimtRows, 0, st>>>(s);
+  mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   dim3 gq((N + fa::kSimtRows - 1) / fa::kSimtRows, B * H);
   fa::bwd_dq_f32_kernel<D><<<gq, 32 * fa::kSimtRows, 0, st>>>(s);
@@ -222,6 +238,11 @@ fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, co
 extern "C" {
 
 int fa_version(void) { return kAbiVersion; }
+
+void fa_set_timing_events(void* start, void* stop) {
+  g_ev_start = static_cast<cudaEvent_t>(start);
+  g_ev_stop = static_cast<cudaEvent_t>(stop);
+}
 
 const char* fa_status_string(fa_status s) {
   switch (s) {

@@ -283,8 +283,11 @@ __global__ void __launch_bounds__(320, 1)
       for (int c = 0; c < 64; ++c) {
         const float p0 = fast_exp2(fmaf(s[2 * c], sl2, -ms));
         const float p1 = fast_exp2(fmaf(s[2 * c + 1], sl2, -ms));
-        rs += p0 + p1;
         pk[c] = pack_bf16x2(p0, p1);
+        // l sums the bf16-rounded weights the P V product actually uses, so the
+        // final O = sum(p v) / l is a convex combination of V rows even when
+        // one key dominates the row.
+        rs += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
       }
       l += rs;
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));

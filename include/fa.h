@@ -102,6 +102,16 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
  */
 fa_status fa_last_device_status(void* stream);
 
+/*
+ * Optional timing hook for benchmarks (off by default).  While both events are
+ * non-NULL, every later fa_fwd / fa_bwd call records `start` on its stream just
+ * before its main attention kernel and `stop` just after it (the forward
+ * kernel; for fa_bwd the tile-recomputing kernel, not the row-term preprocess
+ * or the dQ conversion).  Arguments are cudaEvent_t passed as void*; pass NULLs
+ * to switch it off.  Process-wide and not thread-safe.
+ */
+void fa_set_timing_events(void* start, void* stop);
+
 /* Static, NUL-terminated description of a status code. */
 const char* fa_status_string(fa_status s);
 

@@ -21,7 +21,7 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version"):
+              "fa_version", "fa_set_timing_events"):
         assert n in names
 
 
