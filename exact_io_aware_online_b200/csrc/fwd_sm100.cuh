@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tS = tmem + lane_off + t * 128;
     const uint32_t tO = tmem + lane_off + 256 + t * D;
     const float sl2 = p.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
+    float m_used = -INFINITY, l = 0.f, lb = 0.f;
     bool ok = true;
     for (int jj = 0; jj < nkv; ++jj) {
       const int kv0 = (jlo + jj) * 128;
@@ -263,6 +263,7 @@ __global__ void __launch_bounds__(320, 1)
         const float alpha = need ? fast_exp2(m_used - m_new) : 1.f;
         if (need) {
           l *= alpha;
+          lb *= alpha;
           m_used = m_new;
         }
 #pragma unroll 1
@@ -277,19 +278,21 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_st();
       }
       const float ms = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f;
+      float rs = 0.f, rsb = 0.f;
       uint32_t pk[64];
 #pragma unroll
       for (int c = 0; c < 64; ++c) {
         const float p0 = fast_exp2(fmaf(s[2 * c], sl2, -ms));
         const float p1 = fast_exp2(fmaf(s[2 * c + 1], sl2, -ms));
         pk[c] = pack_bf16x2(p0, p1);
-        // l sums the bf16-rounded weights the P V product actually uses, so the
-        // final O = sum(p v) / l is a convex combination of V rows even when
-        // one key dominates the row.
-        rs += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+        rs += p0 + p1;
+        // lb sums the bf16-rounded weights the P V product actually uses, so
+        // O = sum(p v) / lb is a convex combination of V rows even when one key
+        // dominates the row; l (exact fp32 weights) gives the logsumexp.
+        rsb += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
       }
       l += rs;
+      lb += rsb;
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
       tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
@@ -299,7 +302,7 @@ __global__ void __launch_bounds__(320, 1)
     if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag);
     if (ok) {
       tc_fence_after();
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv = (lb > 0.f) ? 1.f / lb : 0.f;
       uint8_t* sO = sQ + t * C::kTileBytes;  // Q_t is no longer read
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
