@@ -115,29 +115,6 @@ class ClockSampler:
                 "samples": len(self.rows), "power_w_max": max(power) if power else None}
 
 
-def _cudart():
-    import ctypes
-    for name in ("libcudart.so.12", "libcudart.so"):
-        try:
-            lib = ctypes.CDLL(name)
-            lib.cudaEventElapsedTime.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_void_p, ctypes.c_void_p]
-            return lib
-        except OSError:
-            continue
-    raise RuntimeError("libcudart not found")
-
-
-def event_ms(a, b) -> float:
-    """Elapsed ms between two torch events recorded by the C library (torch's
-    own elapsed_time() only accepts events that torch itself recorded)."""
-    import ctypes
-    out = ctypes.c_float(0.0)
-    rc = _cudart().cudaEventElapsedTime(ctypes.byref(out), ctypes.c_void_p(a.cuda_event), ctypes.c_void_p(b.cuda_event))
-    if rc != 0:
-        raise RuntimeError(f"cudaEventElapsedTime failed ({rc})")
-    return float(out.value)
-
-
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -278,6 +255,11 @@ def run_ours(args, w, world, rank, local):
             import torch.distributed as dist
             dist.barrier()
 
+    # torch creates an event's CUDA handle lazily, on its first record():
+    # record each once so the library receives real handles.
+    for a, b in ev_f + ev_b:
+        a.record()
+        b.record()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -297,8 +279,8 @@ def run_ours(args, w, world, rank, local):
     if fa.device_status() != 0:
         raise RuntimeError("device-side timeout during the timed region")
     ms = t_start.elapsed_time(t_stop)
-    fwd_ms = [event_ms(a, b) for a, b in ev_f]
-    bwd_ms = [event_ms(a, b) for a, b in ev_b]
+    fwd_ms = [a.elapsed_time(b) for a, b in ev_f]
+    bwd_ms = [a.elapsed_time(b) for a, b in ev_b]
     if world > 1:
         import torch.distributed as dist
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
