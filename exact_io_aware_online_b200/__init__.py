@@ -14,7 +14,7 @@ import os
 import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
-           "exported_names", "set_timing_events", "LIB_PATH", "HEADER_PATH"]
+           "exported_names", "set_timing_events", "bwd_noalloc", "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -62,6 +62,8 @@ def lib() -> ctypes.CDLL:
     L.fa_version.restype = i
     L.fa_set_timing_events.argtypes = [vp, vp]
     L.fa_set_timing_events.restype = None
+    L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
+    L.fa_bwd_noalloc.restype = i
     _lib = L
     return L
 
@@ -123,6 +125,24 @@ def bwd(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, w
                         B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), code_t,
                         _stream_ptr(q.device))
     _check(code, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_noalloc(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = -1,
+                grads=None):
+    """bwd() for callers that cannot allocate device memory: the library's
+    built-in scratch array replaces the workspace (see fa_bwd_noalloc in fa.h).
+    Pass preallocated `grads`=(dq, dk, dv) to keep the call allocation-free."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    code = lib().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
+                                _stream_ptr(q.device))
+    _check(code, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -305,3 +305,45 @@ fa_status fa_last_device_status(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- fa_bwd_noalloc
+// Scratch for callers that cannot allocate: one file-scope device array per GPU
+// that loads this library.  Host code must not pass `g_bwd_scratch` itself to a
+// kernel (in host code it names a host-side shadow); its device address comes
+// from cudaGetSymbolAddress, looked up once per device and cached.
+namespace {
+
+static __device__ __align__(256) unsigned char g_bwd_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+fa_status noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_bwd_scratch) != cudaSuccess || p == nullptr) return FA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                    const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N,
+                                    int d, float scale, int causal, int window, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (ws_layout(B, H, N, d, dtype).total > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  s = noalloc_scratch(&scratch);
+  if (s != FA_OK) return s;
+  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scratch, FA_BWD_NOALLOC_SCRATCH_BYTES, B, H, Hkv, N, d, scale,
+                causal, window, dtype, stream);
+}

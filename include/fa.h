@@ -96,6 +96,38 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  fa_dtype dtype, void* stream);
 
 /*
+ * Size of the built-in scratch buffer used by fa_bwd_noalloc (16 MiB).
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/*
+ * fa_bwd without a caller-supplied workspace.  (The pages have no counterpart:
+ * this exists for callers, not for the method.)  Some callers cannot allocate
+ * device memory at all -- a plugin running inside a host application that owns
+ * every device allocation and hands the plugin no allocator, or a latency-bound
+ * loop in which a cudaMalloc, which may synchronise the device, is forbidden.
+ * They still pass q, k, v, o, dout, lse and the dq/dk/dv outputs exactly as for
+ * fa_bwd; the scratch fa_bwd would take from `workspace` comes instead from one
+ * file-scope device array of FA_BWD_NOALLOC_SCRATCH_BYTES bytes that every GPU
+ * which loads libfa.so holds until the process exits.  Nothing here calls
+ * cudaMalloc, cudaFree or any allocating routine.
+ *  - Limit: problems whose fa_bwd_workspace_size() exceeds
+ *    FA_BWD_NOALLOC_SCRATCH_BYTES are rejected with FA_ERR_WORKSPACE before
+ *    anything is enqueued (e.g. bf16, d = 128: B*H*ceil(N/128)*128 <= 32256).
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls on a device share the one array and leave their contents in
+ *    it (each call clears what must start at zero itself); calls that can
+ *    overlap on the GPU -- different streams without ordering between them --
+ *    race on it and must be serialised by the caller.
+ * Other arguments, layouts and errors as fa_bwd.
+ */
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, int B, int H, int Hkv, int N, int d,
+                         float scale, int causal, int window, fa_dtype dtype, void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word:
  * FA_ERR_TIMEOUT if a kernel's bounded wait gave up since the last call,
  * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK.
