@@ -18,20 +18,25 @@
 //                    once, dQ partial tiles are added into the accumulator;
 //   bwd_dq_kernel    dQ = bf16(scale * accumulator).
 //
-// Main-kernel roles (320 threads):
-//   warps 0-3  P / dS: one thread per key row (TMEM lanes 0-127)
-//   warps 4-7  dQ drain (one thread per query row of the dQ tile) and the
+// Main-kernel roles (448 threads):
+//   warps 0-3  P / dS for query columns 0-63 of the tile, one thread per key
+//              row (TMEM lanes 0-127)
+//   warps 4-7  the same for query columns 64-127
+//   warps 8-11 dQ drain (one thread per query row of the dQ tile) and the
 //              final dK/dV epilogue (one thread per key row)
-//   warp 8     tcgen05.mma issuer and TMEM owner
-//   warp 9     TMA producer
+//   warp 12    tcgen05.mma issuer and TMEM owner
+//   warp 13    TMA producer (tiles of Q and dO, and the tile's LSE / D rows)
 // The products are formed transposed (S^T = K Q^T, dP^T = V dO^T) so that P^T
 // and dS^T land in TMEM with one key row per lane and can be fed back, as
 // packed bf16, as the A operand of dV += P^T dO and dK += dS^T Q.  dS itself
 // (needed with queries as rows for dQ = dS K) is written to shared memory in
 // the MN-major layout the tensor core reads.
-// TMEM: S^T [0,128) (P^T packed over [0,64)), dP^T [128,256) (dS^T packed over
-// [128,192)), dV [256,256+D), dK [256+D,256+2D); the dQ tile takes [128,256)
-// for D = 128 (after dS^T has been consumed) and [384,448) for D = 64.
+// TMEM: S^T [0,128), dP^T [128,256), dV [256,256+D), dK [256+D,256+2D); the dQ
+// tile takes [128,256) for D = 128 (after dS^T has been consumed) and
+// [384,448) for D = 64.  Each compute warpgroup writes its 64 packed-bf16
+// P^T (dS^T) values per row over the first half of its own 64 S^T (dP^T)
+// columns, so query column c of the tile lives at packed column
+// (c / 64) * 64 + (c % 64) / 2.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -50,16 +55,22 @@ struct BwdParams {
   float scale, scale_log2;
   int causal, window;
   int ntiles;  // Np / 128
+  int group;   // kv heads per rasterisation group (kept L2-resident together)
 };
 
 template <int D>
 struct BwdCfg {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kChunks = D / 64;
-  static constexpr int kStages = (D == 128) ? 2 : 3;  // (Q, dO) tile pairs in flight
+  static constexpr int kStages = (D == 128) ? 2 : 3;  // (Q, dO, LSE, D) tile sets in flight
   static constexpr int kDsBytes = 128 * 128 * 2;
+  static constexpr int kVecBytes = 2 * 128 * 4;       // LSE*log2(e) and D of one query tile
   static constexpr int kNumBars = 1 + 2 * kStages + 8;
-  static constexpr int kSmemBytes = 1024 + 2 * kTileBytes + kStages * 2 * kTileBytes + kDsBytes + 8 * kNumBars + 16;
+  // The dynamic shared window starts 1024-byte aligned (checked at run time),
+  // so no alignment slack is reserved: at D = 128 this fits 227 KB exactly.
+  static constexpr int kSmemBytes =
+      2 * kTileBytes + kStages * 2 * kTileBytes + kDsBytes + kStages * kVecBytes + 8 * kNumBars + 16;
+  static constexpr int kThreads = 448;
   static constexpr bool kAliasDq = (D == 128);
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static constexpr uint32_t kColDQ = kAliasDq ? 128 : 256 + 2 * D;
@@ -139,20 +150,23 @@ __device__ __forceinline__ void stage_row32_bf16(uint8_t* tile, int r, int c, co
 
 // ---------------------------------------------------------------- main kernel
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                      const BwdParams p) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  uint8_t* base = smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr);
-  uint8_t* sK = base;
-  uint8_t* sV = base + C::kTileBytes;
-  uint8_t* sStage = base + 2 * C::kTileBytes;  // stage s: Q at +0, dO at +kTileBytes
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {  // layout below assumes a 1024-aligned window
+    if (threadIdx.x == 0) atomicOr(&g_status, kStatusMisaligned);
+    return;
+  }
+  uint8_t* sK = smem_raw;
+  uint8_t* sV = smem_raw + C::kTileBytes;
+  uint8_t* sStage = smem_raw + 2 * C::kTileBytes;  // stage s: Q at +0, dO at +kTileBytes
   uint8_t* sDS = sStage + C::kStages * 2 * C::kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + C::kDsBytes);
+  uint8_t* sVec = sDS + C::kDsBytes;  // stage s: LSE*log2(e) [128] then D [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sVec + C::kStages * C::kVecBytes);
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
   uint64_t* q_empty = bars + 1 + C::kStages;
@@ -169,10 +183,17 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work unit: key tile j of kv head (b, kh); small j (most query tiles under a causal mask) first
+  // ---- work unit: key tile j of kv head bkv.  Groups of p.group kv heads run
+  // together (their Q, dO, K, V and dQ accumulator stay in L2); inside a group
+  // the smallest j (the most query tiles under a causal mask) goes first.
   const int BHkv = p.B * p.Hkv;
-  const int j = static_cast<int>(blockIdx.x) / BHkv;
-  const int bkv = static_cast<int>(blockIdx.x) % BHkv;
+  const int per_group = p.group * p.ntiles;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int g0 = grp * p.group;
+  const int gsz = min(p.group, BHkv - g0);
+  const int rem = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int j = rem / gsz;
+  const int bkv = g0 + rem % gsz;
   const int b = bkv / p.Hkv, kh = bkv % p.Hkv;
   const int k0 = j * 128;
   int ilo = 0, ihi = p.ntiles - 1;
@@ -194,8 +215,8 @@ __global__ void __launch_bounds__(320, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(ds_full, 128);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
     mbar_init(kv_done, 1);
@@ -203,7 +224,7 @@ __global__ void __launch_bounds__(320, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
     tc_fence_before();
@@ -212,7 +233,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 9) {
+  if (warp == 13) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
@@ -230,13 +251,16 @@ __global__ void __launch_bounds__(320, 1)
       for (int it = 0; it < total; ++it) {
         const int s = it % C::kStages;
         if (!mbar_wait(&q_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&q_full[s], 2 * C::kTileBytes);
+        mbar_arrive_expect_tx(&q_full[s], 2 * C::kTileBytes + C::kVecBytes);
         const int row0 = q_tile(it) * 128, bh = q_head(it);
         uint8_t* st = sStage + s * 2 * C::kTileBytes;
         for (int c = 0; c < C::kChunks; ++c) {
           tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
           tma_load_3d(&tmdO, &q_full[s], st + C::kTileBytes + c * 16384, c * 64, row0, bh);
         }
+        const size_t vrow = static_cast<size_t>(bh) * p.Np + row0;
+        bulk_load(sVec + s * C::kVecBytes, p.lse2 + vrow, 512, &q_full[s]);
+        bulk_load(sVec + s * C::kVecBytes + 512, p.Drow + vrow, 512, &q_full[s]);
         ++issued[s];
       }
       const unsigned long long t0 = globaltimer_ns();
@@ -248,7 +272,7 @@ __global__ void __launch_bounds__(320, 1)
                  globaltimer_ns() - t0 < kWaitLimitNs) {
           }
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aSt = smem_u32(sStage), aDS = smem_u32(sDS);
@@ -265,11 +289,12 @@ __global__ void __launch_bounds__(320, 1)
           umma_ss(tmem + dcol, sdesc_sw128(a + off, 16, 1024), sdesc_sw128(bb + off, 16, 1024), kIdS, k > 0);
         }
       };
-      // acc += X^T(tmem, packed bf16, 128 keys x 128 queries) * B(smem, queries x D, MN-major)
+      // acc += X^T(tmem, packed bf16, keys x queries) * B(smem, queries x D, MN-major)
       auto ts_acc = [&](uint32_t dcol, uint32_t acol, uint32_t bb, bool acc) {
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          umma_ts(tmem + dcol, tmem + acol + k * 8, sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
+          umma_ts(tmem + dcol, tmem + acol + (k >> 2) * 64 + (k & 3) * 8,
+                  sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&q_full[0], 0, abort_flag);
       if (ok) {
@@ -316,56 +341,55 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) umma_commit(kv_done);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ------------------------------------------------------------ P and dS (one key row per thread)
-    const int r = warp * 32 + lane;
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P and dS
+    // Warpgroup w handles query columns [64w, 64w + 64); one key row per thread.
+    const int w = warp >> 2, wl = warp & 3;
+    const int r = wl * 32 + lane;
     const int key = k0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::kColS;
-    const uint32_t tDP = tmem + lane_off + C::kColDP;
+    const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::kColS + 64 * w;
+    const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * w;
     const float sl2 = p.scale_log2;
+    const int ds_chunk = w;  // 64-column (128-byte) block of the dS tile
     bool ok = true;
     for (int it = 0; it < total; ++it) {
-      const int i = q_tile(it);
-      const int q0 = i * 128;
-      const size_t vrow = static_cast<size_t>(q_head(it)) * p.Np + q0;
-      const float4* L4 = reinterpret_cast<const float4*>(p.lse2 + vrow);
-      const float4* D4 = reinterpret_cast<const float4*>(p.Drow + vrow);
-      bool full = true;  // every (query, key) pair of the tile allowed?
+      const int s = it % C::kStages;
+      const int q0 = q_tile(it) * 128 + 64 * w;  // first query of my columns
+      const float4* L4 = reinterpret_cast<const float4*>(sVec + s * C::kVecBytes) + 16 * w;
+      const float4* D4 = reinterpret_cast<const float4*>(sVec + s * C::kVecBytes + 512) + 16 * w;
+      bool full = true;  // every (query, key) pair of my 64 columns allowed?
       if (p.causal) full = full && (k0 + 127 <= q0);
-      if (p.window >= 0) full = full && (q0 + 127 - k0 <= p.window) && (k0 + 127 - q0 <= p.window);
+      if (p.window >= 0) full = full && (q0 + 63 - k0 <= p.window) && (k0 + 127 - q0 <= p.window);
+      if (!(ok = mbar_wait(&q_full[s], (it / C::kStages) & 1, abort_flag))) break;  // LSE / D landed
       if (!(ok = mbar_wait(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      uint32_t pk[64];  // P^T row, packed bf16
+      uint32_t sv[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_wait_ld();
+      uint32_t pk[32];  // my 64 P^T values, packed bf16
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32];
-        tmem_ld32(tS + c * 32, sv);
-        tmem_wait_ld();
+      for (int u = 0; u < 16; ++u) {
+        const float4 l4 = L4[u];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        float pv[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 l4 = __ldg(&L4[c * 8 + u]);
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-          float pv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int qc = c * 32 + u * 4 + e;
-            float x = fast_exp2(fmaf(__uint_as_float(sv[u * 4 + e]), sl2, -lv[e]));
-            if (!full) {
-              const int q = q0 + qc;
-              bool keep = true;
-              if (p.causal) keep = keep && key <= q;
-              if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
-              if (!keep) x = 0.f;
-            }
-            pv[e] = x;
+        for (int e = 0; e < 4; ++e) {
+          float x = fast_exp2(fmaf(__uint_as_float(sv[u * 4 + e]), sl2, -lv[e]));
+          if (!full) {
+            const int q = q0 + u * 4 + e;
+            bool keep = true;
+            if (p.causal) keep = keep && key <= q;
+            if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
+            if (!keep) x = 0.f;
           }
-          pk[c * 16 + u * 2 + 0] = pack_bf16x2(pv[0], pv[1]);
-          pk[c * 16 + u * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+          pv[e] = x;
         }
+        pk[u * 2 + 0] = pack_bf16x2(pv[0], pv[1]);
+        pk[u * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
       }
-      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st32(tS, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
@@ -373,33 +397,32 @@ __global__ void __launch_bounds__(320, 1)
       if (!(ok = mbar_wait(dp_full, it & 1, abort_flag))) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int h = 0; h < 2; ++h) {
         uint32_t dv[32];
-        tmem_ld32(tDP + c * 32, dv);
+        tmem_ld32(tDP + 32 * h, dv);
         tmem_wait_ld();
         uint32_t ds[16];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const float4 d4 = __ldg(&D4[c * 8 + u]);
+          const float4 d4 = D4[h * 8 + u];
           const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
           for (int e2 = 0; e2 < 2; ++e2) {
-            const __nv_bfloat162 pp = *reinterpret_cast<const __nv_bfloat162*>(&pk[c * 16 + u * 2 + e2]);
-            const float2 pf = __bfloat1622float2(pp);
-            const float g0 = pf.x * (__uint_as_float(dv[u * 4 + e2 * 2 + 0]) - dd[e2 * 2 + 0]);
-            const float g1 = pf.y * (__uint_as_float(dv[u * 4 + e2 * 2 + 1]) - dd[e2 * 2 + 1]);
+            const uint32_t pp = pk[h * 16 + u * 2 + e2];
+            const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
+            const float g0 = p0 * (__uint_as_float(dv[u * 4 + e2 * 2 + 0]) - dd[e2 * 2 + 0]);
+            const float g1 = p1 * (__uint_as_float(dv[u * 4 + e2 * 2 + 1]) - dd[e2 * 2 + 1]);
             ds[u * 2 + e2] = pack_bf16x2(g0, g1);
           }
         }
-        // dS^T (packed) into TMEM over dP^T columns already read; dS into shared
-        // memory as rows = keys, columns = queries (MN-major A operand of dQ).
-        tmem_st16(tDP + c * 16, ds);
-        const int chunk = c >> 1;
-        const int u0 = (c & 1) * 4;
+        // dS^T (packed) over dP^T columns this thread has already read; dS into
+        // shared memory as rows = keys, columns = queries (MN-major A of dQ).
+        tmem_st16(tDP + 16 * h, ds);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          uint4 val = make_uint4(ds[4 * u], ds[4 * u + 1], ds[4 * u + 2], ds[4 * u + 3]);
-          *reinterpret_cast<uint4*>(sDS + chunk * 16384 + r * 128 + (((u0 + u) ^ (r & 7)) << 4)) = val;
+          const int unit = h * 4 + u;  // 16-byte unit within my 128-byte row chunk
+          *reinterpret_cast<uint4*>(sDS + ds_chunk * 16384 + r * 128 + ((unit ^ (r & 7)) << 4)) =
+              make_uint4(ds[4 * u], ds[4 * u + 1], ds[4 * u + 2], ds[4 * u + 3]);
         }
       }
       tmem_wait_st();
@@ -416,16 +439,20 @@ __global__ void __launch_bounds__(320, 1)
     for (int it = 0; it < total; ++it) {
       if (!(ok = mbar_wait(dq_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      uint32_t v[D];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c)
-        tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(dq_empty);
       float* dst = p.dqacc + (static_cast<size_t>(q_head(it)) * p.Np + q_tile(it) * 128 + r) * D;
 #pragma unroll
-      for (int c = 0; c < D; c += 4) red_add_v4(dst + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+      for (int half = 0; half < D / 64; ++half) {
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_off + C::kColDQ + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tmem + lane_off + C::kColDQ + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
+        if (half == D / 64 - 1) {
+          tc_fence_before();
+          mbar_arrive(dq_empty);
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) red_add_v4(dst + half * 64 + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+      }
     }
     if (ok) ok = mbar_wait(kv_done, 0, abort_flag);
     if (ok) {
@@ -455,7 +482,7 @@ __global__ void __launch_bounds__(320, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

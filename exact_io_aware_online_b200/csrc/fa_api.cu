@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -118,6 +119,12 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   p.window = window;
   p.npairs = (N + 255) / 256;
   p.ntiles_kv = (N + 127) / 128;
+  {  // heads per group: Q, O and the (shared) K, V of a group within ~64 MiB of L2
+    const double unit = static_cast<double>(N) * D * (4.0 + 4.0 / p.g);
+    p.group = std::min(B * H, static_cast<int>(std::max(1.0, std::floor((64.0 * 1024 * 1024) / unit))));
+    p.group = std::max(p.g, p.group / p.g * p.g);  // whole GQA groups
+    p.group = std::min(p.group, B * H);
+  }
   const unsigned grid = static_cast<unsigned>(p.npairs) * B * H;
   mark_start(st);
   fa::fwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
@@ -185,6 +192,13 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   p.causal = causal ? 1 : 0;
   p.window = window;
   p.ntiles = p.Np / 128;
+  // kv heads per rasterisation group: keep each group's Q, dO, K, V and dQ
+  // accumulator (about N*d*(4 + 8g) bytes per kv head) within ~64 MiB of L2.
+  {
+    const double unit = static_cast<double>(p.Np) * D * (4.0 + 8.0 * p.g);
+    p.group = static_cast<int>(std::max(1.0, std::floor((64.0 * 1024 * 1024) / unit)));
+    p.group = std::min(p.group, B * Hkv);
+  }
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if (!make_tile_map(&tq, q, B * H, N, D) || !make_tile_map(&tk, k, B * Hkv, N, D) ||
       !make_tile_map(&tv, v, B * Hkv, N, D) || !make_tile_map(&tdo, dout, B * H, N, D) ||
@@ -196,7 +210,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   if (launched() != FA_OK) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.ntiles) * B * Hkv;
   mark_start(st);
-  fa::bwd_sm100_kernel<D><<<grid, 320, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
+  fa::bwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   const size_t n4 = static_cast<size_t>(B) * H * N * D / 4;
@@ -301,7 +315,8 @@ fa_status fa_last_device_status(void* stream) {
   unsigned int v = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&v, fa::g_status, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(fa::g_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
-  return (v & fa::kStatusTimeout) ? FA_ERR_TIMEOUT : FA_OK;
+  if (v & fa::kStatusTimeout) return FA_ERR_TIMEOUT;
+  return v ? FA_ERR_CUDA : FA_OK;
 }
 
 }  // extern "C"

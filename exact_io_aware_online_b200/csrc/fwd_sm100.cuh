@@ -36,6 +36,7 @@ struct FwdParams {
   int causal, window;
   int npairs;     // ceil(N / 256): query-tile pairs per head
   int ntiles_kv;  // ceil(N / 128)
+  int group;      // heads per rasterisation group (kept L2-resident together)
 };
 
 template <int D>
@@ -78,10 +79,17 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work unit: heaviest (last) query-tile pairs first
+  // ---- work unit: query-tile pair `pair` of head bh.  Groups of p.group heads
+  // run together (their K/V stay in L2); inside a group the heaviest (last)
+  // pairs under a causal mask go first.
   const int BH = p.B * p.H;
-  const int pair = p.npairs - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int per_group = p.group * p.npairs;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int g0 = grp * p.group;
+  const int gsz = min(p.group, BH - g0);
+  const int rem = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int pair = p.npairs - 1 - rem / gsz;
+  const int bh = g0 + rem % gsz;
   const int b = bh / p.H, h = bh % p.H;
   const int kvh = b * p.Hkv + h / p.g;
   const int q0 = pair * 256;

@@ -13,6 +13,7 @@ namespace fa {
 // Device status word: a bounded wait that gives up ORs a code in here.
 __device__ unsigned int g_status;
 constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusMisaligned = 2u;  // dynamic shared memory not 1024-byte aligned
 // About two seconds: long enough for any legitimate wait, short enough that a
 // protocol bug ends the kernel instead of hanging the GPU.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
@@ -81,6 +82,13 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* ba
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+}
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
