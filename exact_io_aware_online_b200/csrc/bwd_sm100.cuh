@@ -18,14 +18,21 @@
 //                    once, dQ partial tiles are added into the accumulator;
 //   bwd_dq_kernel    dQ = bf16(scale * accumulator).
 //
-// Main-kernel roles (448 threads):
-//   warps 0-3  P / dS for query columns 0-63 of the tile, one thread per key
-//              row (TMEM lanes 0-127)
-//   warps 4-7  the same for query columns 64-127
-//   warps 8-11 dQ drain (one thread per query row of the dQ tile) and the
-//              final dK/dV epilogue (one thread per key row)
-//   warp 12    tcgen05.mma issuer and TMEM owner
-//   warp 13    TMA producer (tiles of Q and dO, and the tile's LSE / D rows)
+// Main-kernel roles (512 threads, four warpgroups):
+//   warps 0-3   P / dS for query columns 0-63 of the tile, one thread per key
+//               row (TMEM lanes 0-127)
+//   warps 4-7   the same for query columns 64-127
+//   warps 8-11  dQ drain (one thread per query row of the dQ tile) and the
+//               final dK/dV epilogue (one thread per key row)
+//   warp 12     tcgen05.mma issuer and TMEM owner
+//   warp 13     TMA producer (tiles of Q and dO, and the tile's LSE / D rows)
+//   warps 14-15 idle (they complete the fourth warpgroup)
+// Registers: 128 per thread at launch; the fourth warpgroup gives up 72 and
+// the drain takes them (128 + 128 + 200 + 56 = 4 * 128), so a drain thread
+// holds a whole dQ row and releases the TMEM tile before its reductions.
+// The dQ accumulator uses a lane-interleaved layout (see dqacc_index) so that
+// the drain's vector reductions are coalesced: one warp instruction adds 512
+// contiguous bytes instead of touching 32 rows.
 // The products are formed transposed (S^T = K Q^T, dP^T = V dO^T) so that P^T
 // and dS^T land in TMEM with one key row per lane and can be fed back, as
 // packed bf16, as the A operand of dV += P^T dO and dK += dS^T Q.  dS itself
@@ -70,7 +77,7 @@ struct BwdCfg {
   // so no alignment slack is reserved: at D = 128 this fits 227 KB exactly.
   static constexpr int kSmemBytes =
       2 * kTileBytes + kStages * 2 * kTileBytes + kDsBytes + kStages * kVecBytes + 8 * kNumBars + 16;
-  static constexpr int kThreads = 448;
+  static constexpr int kThreads = 512;
   static constexpr bool kAliasDq = (D == 128);
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static constexpr uint32_t kColDQ = kAliasDq ? 128 : 256 + 2 * D;
@@ -111,20 +118,50 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   }
 }
 
+// ---------------------------------------------------------------- dQ accumulator layout
+// Rows are taken in groups of 32 (row n = 32 g + l).  Inside a group, the
+// 16-byte unit u (columns 4u..4u+3) of the 32 rows is stored contiguously, row
+// l at offset 16 l: element (n, c) of head bh sits at float index
+//   ((bh * Np/32 + g) * D/4 + c/4) * 128 + 4 l + c % 4.
+// A warp whose lane l owns row 32 g + l then adds unit u of all 32 rows with
+// one coalesced 512-byte vector reduction.
+template <int D>
+__device__ __forceinline__ size_t dqacc_unit(size_t bh, int Np, int g, int u) {
+  return ((bh * static_cast<size_t>(Np / 32) + g) * (D / 4) + u) * 128;
+}
+
 // ---------------------------------------------------------------- dQ convert
+// One block per 32-row group: coalesced reads of the interleaved accumulator,
+// a transpose through shared memory, coalesced bf16 row writes of scale * acc.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
-  const size_t i4 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // float4 index
-  const size_t total4 = static_cast<size_t>(p.B) * p.H * p.N * D / 4;
-  if (i4 >= total4) return;
-  const size_t e = i4 * 4;
-  const size_t row = e / D, col = e % D;
-  const size_t bh = row / p.N, n = row % p.N;
-  const float4 a = *reinterpret_cast<const float4*>(p.dqacc + (bh * p.Np + n) * D + col);
-  uint2 out;
-  out.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
-  out.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
-  *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + e) = out;
+  __shared__ float tile[32][D + 4];
+  const int groups = p.Np / 32;
+  const size_t bh = blockIdx.x / groups;
+  const int g = static_cast<int>(blockIdx.x % groups);
+  const float4* src = reinterpret_cast<const float4*>(p.dqacc + dqacc_unit<D>(bh, p.Np, g, 0));
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) {  // 32 * D / 4 float4 per group, 256 threads
+    const int f = threadIdx.x + 256 * k;
+    const int u = f >> 5, l = f & 31;
+    const float4 a = src[f];
+    tile[l][4 * u + 0] = a.x;
+    tile[l][4 * u + 1] = a.y;
+    tile[l][4 * u + 2] = a.z;
+    tile[l][4 * u + 3] = a.w;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) {
+    const int f = threadIdx.x + 256 * k;
+    const int rr = f / (D / 4), u = f % (D / 4);
+    const int n = 32 * g + rr;
+    if (n >= p.N) continue;
+    uint2 out;
+    out.x = pack_bf16x2(tile[rr][4 * u + 0] * p.scale, tile[rr][4 * u + 1] * p.scale);
+    out.y = pack_bf16x2(tile[rr][4 * u + 2] * p.scale, tile[rr][4 * u + 3] * p.scale);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (bh * p.N + n) * D + 4 * u) = out;
+  }
 }
 
 __device__ __forceinline__ void red_add_v4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -150,7 +187,7 @@ __device__ __forceinline__ void stage_row32_bf16(uint8_t* tile, int r, int c, co
 
 // ---------------------------------------------------------------- main kernel
 template <int D>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
@@ -233,9 +270,10 @@ __global__ void __launch_bounds__(448, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 13) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp >= 12) {
+    regs_dec<56>();
+    if (warp == 13 && lane == 0) {
+      // ---------------------------------------------------------- producer
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
@@ -271,10 +309,8 @@ __global__ void __launch_bounds__(448, 1)
           while (!mbar_try_wait(smem_u32(&q_full[s]), (issued[s] - 1) & 1) &&
                  globaltimer_ns() - t0 < kWaitLimitNs) {
           }
-    }
-  } else if (warp == 12) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 12 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aSt = smem_u32(sStage), aDS = smem_u32(sDS);
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, false, true);     // dV, dK (A from TMEM)
@@ -356,8 +392,8 @@ __global__ void __launch_bounds__(448, 1)
     for (int it = 0; it < total; ++it) {
       const int s = it % C::kStages;
       const int q0 = q_tile(it) * 128 + 64 * w;  // first query of my columns
-      const float4* L4 = reinterpret_cast<const float4*>(sVec + s * C::kVecBytes) + 16 * w;
-      const float4* D4 = reinterpret_cast<const float4*>(sVec + s * C::kVecBytes + 512) + 16 * w;
+      const float* Lv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes) + 64 * w;
+      const float* Dv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes + 512) + 64 * w;
       bool full = true;  // every (query, key) pair of my 64 columns allowed?
       if (p.causal) full = full && (k0 + 127 <= q0);
       if (p.window >= 0) full = full && (q0 + 63 - k0 <= p.window) && (k0 + 127 - q0 <= p.window);
@@ -368,27 +404,25 @@ __global__ void __launch_bounds__(448, 1)
       tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
+      float pv[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float lv = Lv[c];
+        pv[c] = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -lv));
+      }
+      if (!full) {  // tiles on the diagonal / window edge only: one branch, not one per element
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          const int q = q0 + c;
+          bool keep = true;
+          if (p.causal) keep = keep && key <= q;
+          if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
+          pv[c] = keep ? pv[c] : 0.f;
+        }
+      }
       uint32_t pk[32];  // my 64 P^T values, packed bf16
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const float4 l4 = L4[u];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-        float pv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float x = fast_exp2(fmaf(__uint_as_float(sv[u * 4 + e]), sl2, -lv[e]));
-          if (!full) {
-            const int q = q0 + u * 4 + e;
-            bool keep = true;
-            if (p.causal) keep = keep && key <= q;
-            if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
-            if (!keep) x = 0.f;
-          }
-          pv[e] = x;
-        }
-        pk[u * 2 + 0] = pack_bf16x2(pv[0], pv[1]);
-        pk[u * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-      }
+      for (int u = 0; u < 32; ++u) pk[u] = pack_bf16x2(pv[2 * u], pv[2 * u + 1]);
       tmem_st32(tS, pk);
       tmem_wait_st();
       tc_fence_before();
@@ -403,17 +437,11 @@ __global__ void __launch_bounds__(448, 1)
         tmem_wait_ld();
         uint32_t ds[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float4 d4 = D4[h * 8 + u];
-          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const uint32_t pp = pk[h * 16 + u * 2 + e2];
-            const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
-            const float g0 = p0 * (__uint_as_float(dv[u * 4 + e2 * 2 + 0]) - dd[e2 * 2 + 0]);
-            const float g1 = p1 * (__uint_as_float(dv[u * 4 + e2 * 2 + 1]) - dd[e2 * 2 + 1]);
-            ds[u * 2 + e2] = pack_bf16x2(g0, g1);
-          }
+        for (int u = 0; u < 16; ++u) {
+          const uint32_t pp = pk[h * 16 + u];
+          const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
+          const float d0 = Dv[32 * h + 2 * u], d1 = Dv[32 * h + 2 * u + 1];
+          ds[u] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * u]) - d0), p1 * (__uint_as_float(dv[2 * u + 1]) - d1));
         }
         // dS^T (packed) over dP^T columns this thread has already read; dS into
         // shared memory as rows = keys, columns = queries (MN-major A of dQ).
@@ -432,6 +460,7 @@ __global__ void __launch_bounds__(448, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ drain, then dK/dV epilogue
+    regs_inc<200>();
     const int wl = warp & 3;
     const int r = wl * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
@@ -439,20 +468,17 @@ __global__ void __launch_bounds__(448, 1)
     for (int it = 0; it < total; ++it) {
       if (!(ok = mbar_wait(dq_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      float* dst = p.dqacc + (static_cast<size_t>(q_head(it)) * p.Np + q_tile(it) * 128 + r) * D;
+      // my row is 32 * (4 * q_tile + wl) + lane: group 4 * q_tile + wl, slot `lane`
+      float* dst = p.dqacc + dqacc_unit<D>(q_head(it), p.Np, 4 * q_tile(it) + wl, 0) + 4 * lane;
+      uint32_t v[D];
 #pragma unroll
-      for (int half = 0; half < D / 64; ++half) {
-        uint32_t v[64];
-        tmem_ld32(tmem + lane_off + C::kColDQ + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-        tmem_ld32(tmem + lane_off + C::kColDQ + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
-        tmem_wait_ld();
-        if (half == D / 64 - 1) {
-          tc_fence_before();
-          mbar_arrive(dq_empty);
-        }
+      for (int c = 0; c < D / 32; ++c)
+        tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(dq_empty);  // TMEM tile free before the reductions are issued
 #pragma unroll
-        for (int c = 0; c < 64; c += 4) red_add_v4(dst + half * 64 + c, v[c], v[c + 1], v[c + 2], v[c + 3]);
-      }
+      for (int c = 0; c < D; c += 4) red_add_v4(dst + 32 * c, v[c], v[c + 1], v[c + 2], v[c + 3]);
     }
     if (ok) ok = mbar_wait(kv_done, 0, abort_flag);
     if (ok) {

@@ -213,8 +213,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   fa::bwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
-  const size_t n4 = static_cast<size_t>(B) * H * N * D / 4;
-  fa::bwd_dq_kernel<D><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(p);
+  fa::bwd_dq_kernel<D><<<static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32)), 256, 0, st>>>(p);
   return launched();
 }
 
