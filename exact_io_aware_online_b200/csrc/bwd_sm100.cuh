@@ -27,8 +27,8 @@
 //   warp 12     tcgen05.mma issuer and TMEM owner
 //   warp 13     TMA producer (tiles of Q and dO, and the tile's LSE / D rows)
 //   warps 14-15 idle (they complete the fourth warpgroup)
-// Registers: 128 per thread at launch; the fourth warpgroup gives up 72 and
-// the drain takes them (128 + 128 + 200 + 56 = 4 * 128), so a drain thread
+// Registers: 128 per thread at launch; the fourth warpgroup gives up 56 and
+// the drain takes them (128 + 128 + 184 + 72 = 4 * 128), so a drain thread
 // holds a whole dQ row and releases the TMEM tile before its reductions.
 // The dQ accumulator uses a lane-interleaved layout (see dqacc_index) so that
 // the drain's vector reductions are coalesced: one warp instruction adds 512
@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 12) {
-    regs_dec<56>();
+    regs_dec<72>();
     if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- producer
       prefetch_tmap(&tmQ);
@@ -460,7 +460,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ drain, then dK/dV epilogue
-    regs_inc<200>();
+    regs_inc<184>();
     const int wl = warp & 3;
     const int r = wl * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;

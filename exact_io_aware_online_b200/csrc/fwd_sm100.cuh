@@ -9,11 +9,15 @@
 // block at a time).  Only O and the logsumexp reach global memory ("FlashAttention"
 // guide page, "Tiling through SRAM").
 //
-// Roles (320 threads):
-//   warps 0-3  softmax for query tile 0, one thread per row (TMEM lanes 0-127)
-//   warps 4-7  softmax for query tile 1
-//   warp 8     tcgen05.mma issuer (one thread) and TMEM owner
-//   warp 9     TMA producer (one thread)
+// Roles (384 threads, three warpgroups):
+//   warps 0-3   softmax for query tile 0, one thread per row (TMEM lanes 0-127)
+//   warps 4-7   softmax for query tile 1
+//   warp 8      tcgen05.mma issuer (one thread) and TMEM owner
+//   warp 9      TMA producer (one thread)
+//   warps 10-11 idle (they complete the third warpgroup)
+// Registers: 168 per thread at launch; the third warpgroup drops to 72 and the
+// two softmax warpgroups rise to 216 (216 + 216 + 72 = 3 * 168), enough to hold
+// a whole 128-key score row per thread without spilling.
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
 // P_t overwrites S_t as packed bf16 (64 columns) and is the A operand of the
 // P V product straight from TMEM, so P never touches shared memory.
@@ -48,7 +52,7 @@ struct FwdCfg {
   static constexpr int kSmemKV = kStages * kTileBytes;
   static constexpr int kNumBars = 1 + 2 * kStages + 8;
   static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + 8 * kNumBars + 16;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -56,7 +60,7 @@ constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units (factor 256)
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                      const FwdParams p) {
@@ -126,9 +130,10 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 9) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp >= 8) {
+    regs_dec<72>();
+    if (warp == 9 && lane == 0) {
+      // ---------------------------------------------------------- producer
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
@@ -161,10 +166,8 @@ __global__ void __launch_bounds__(320, 1)
           while (!mbar_try_wait(smem_u32(&kv_full[s]), (issued[s] - 1) & 1) &&
                  globaltimer_ns() - t0 < kWaitLimitNs) {
           }
-    }
-  } else if (warp == 8) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 8 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
       const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV);
       constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdescO = idesc_bf16_f32(128, D, false, true);
@@ -222,6 +225,7 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax (tile t)
+    regs_inc<216>();
     const int t = warp >> 2;
     const int wl = warp & 3;
     const int r = wl * 32 + lane;
@@ -257,9 +261,14 @@ __global__ void __launch_bounds__(320, 1)
           if (!keep) s[c] = -INFINITY;
         }
       }
-      float mx = s[0];
+      float mx8[8];  // eight independent partial maxima (short dependency chains)
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+      for (int c = 8; c < 128; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
+      const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmax3(mx8[6], mx8[7], mx8[7])));
       const float m_new = fmaxf(m_used, mx * sl2);
       bool need = false;
       if (m_used == -INFINITY) {
@@ -286,23 +295,34 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_st();
       }
       const float ms = (m_used == -INFINITY) ? 0.f : m_used;
-      float rs = 0.f, rsb = 0.f;
-      uint32_t pk[64];
+      const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
+      // Row sums on packed fp32 pairs, two independent accumulators each.  rs:
+      // exact fp32 weights (gives the logsumexp); rsb: the bf16-rounded weights
+      // the P V product actually uses, so O = sum(p v) / lb is a convex
+      // combination of V rows even when one key dominates the row.
+      uint64_t rs2[2] = {0ull, 0ull}, rsb2[2] = {0ull, 0ull};
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = fast_exp2(fmaf(s[2 * c], sl2, -ms));
-        const float p1 = fast_exp2(fmaf(s[2 * c + 1], sl2, -ms));
-        pk[c] = pack_bf16x2(p0, p1);
-        rs += p0 + p1;
-        // lb sums the bf16-rounded weights the P V product actually uses, so
-        // O = sum(p v) / lb is a convex combination of V rows even when one key
-        // dominates the row; l (exact fp32 weights) gives the logsumexp.
-        rsb += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+      for (int ch = 0; ch < 4; ++ch) {  // 32 keys per chunk, stored as soon as packed
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int c = ch * 32 + 2 * u;
+          float x0, x1;
+          f2_split(ffma2(f2(s[c], s[c + 1]), sl2x2, nmsx2), x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          pk[u] = pack_bf16x2(p0, p1);
+          rs2[u & 1] = fadd2(rs2[u & 1], f2(p0, p1));
+          rsb2[u & 1] = fadd2(rsb2[u & 1], f2(__uint_as_float(pk[u] << 16), __uint_as_float(pk[u] & 0xffff0000u)));
+        }
+        tmem_st16(tS + ch * 16, pk);
       }
-      l += rs;
-      lb += rsb;
-      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      {
+        float a0, a1, b0, b1;
+        f2_split(fadd2(rs2[0], rs2[1]), a0, a1);
+        f2_split(fadd2(rsb2[0], rsb2[1]), b0, b1);
+        l += a0 + a1;
+        lb += b0 + b1;
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
