@@ -59,6 +59,67 @@ struct FwdCfg {
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units (factor 256)
 constexpr float kLn2 = 0.69314718055994530942f;
 
+// 2^x for a pair of values on the FMA pipe.  Cody-Waite reduction x = n + f,
+// n = rint(x) (added to the exponent field), f in [-1/2, 1/2], and the degree-3
+// polynomial with minimal maximum relative error for 2^f on that interval
+// (7.5e-5; coefficients from exp2_poly.py, a Remez exchange).  x is clamped at
+// -126 so the exponent add cannot wrap; callers use it on unmasked tiles only.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t xx = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(xx, f2(kMagic, kMagic));
+  const uint64_t n = fadd2(t, f2(-kMagic, -kMagic));
+  const uint64_t f = ffma2(n, f2(-1.f, -1.f), xx);
+  uint64_t p = ffma2(f, f2(0.05517167f, 0.05517167f), f2(0.24261113f, 0.24261113f));
+  p = ffma2(p, f, f2(0.69326097f, 0.69326097f));
+  p = ffma2(p, f, f2(0.99992806f, 0.99992806f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
+// p = 2^(s * scale_log2 - m) for one 128-key score row, written to TMEM as packed
+// bf16 in four 32-key chunks; accumulates the fp32 row sum (l) and the sum of
+// the bf16-rounded values (lb).  kPoly: one pair in four uses exp2_poly2 so
+// the special-function unit is not the only source of exponentials.
+template <bool kPoly>
+__device__ __forceinline__ void exp_row_to_tmem(const float (&s)[128], float sl2, float ms, uint32_t tS, float& l,
+                                                float& lb) {
+  const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
+  // Row sums on packed fp32 pairs, two independent accumulators each.  rs:
+  // exact fp32 weights (gives the logsumexp); rsb: the bf16-rounded weights
+  // the P V product actually uses, so O = sum(p v) / lb is a convex
+  // combination of V rows even when one key dominates the row.
+  uint64_t rs2[2] = {0ull, 0ull}, rsb2[2] = {0ull, 0ull};
+#pragma unroll
+  for (int ch = 0; ch < 4; ++ch) {  // 32 keys per chunk, stored as soon as packed
+    uint32_t pk[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const int c = ch * 32 + 2 * u;
+      float x0, x1, p0, p1;
+      f2_split(ffma2(f2(s[c], s[c + 1]), sl2x2, nmsx2), x0, x1);
+      if (kPoly && (u & 3) == 3) {
+        exp2_poly2(x0, x1, p0, p1);
+      } else {
+        p0 = fast_exp2(x0);
+        p1 = fast_exp2(x1);
+      }
+      pk[u] = pack_bf16x2(p0, p1);
+      rs2[u & 1] = fadd2(rs2[u & 1], f2(p0, p1));
+      rsb2[u & 1] = fadd2(rsb2[u & 1], f2(__uint_as_float(pk[u] << 16), __uint_as_float(pk[u] & 0xffff0000u)));
+    }
+    tmem_st16(tS + ch * 16, pk);
+  }
+  float a0, a1, b0, b1;
+  f2_split(fadd2(rs2[0], rs2[1]), a0, a1);
+  f2_split(fadd2(rsb2[0], rsb2[1]), b0, b1);
+  l += a0 + a1;
+  lb += b0 + b1;
+}
+
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -295,34 +356,10 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_st();
       }
       const float ms = (m_used == -INFINITY) ? 0.f : m_used;
-      const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
-      // Row sums on packed fp32 pairs, two independent accumulators each.  rs:
-      // exact fp32 weights (gives the logsumexp); rsb: the bf16-rounded weights
-      // the P V product actually uses, so O = sum(p v) / lb is a convex
-      // combination of V rows even when one key dominates the row.
-      uint64_t rs2[2] = {0ull, 0ull}, rsb2[2] = {0ull, 0ull};
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {  // 32 keys per chunk, stored as soon as packed
-        uint32_t pk[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int c = ch * 32 + 2 * u;
-          float x0, x1;
-          f2_split(ffma2(f2(s[c], s[c + 1]), sl2x2, nmsx2), x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          pk[u] = pack_bf16x2(p0, p1);
-          rs2[u & 1] = fadd2(rs2[u & 1], f2(p0, p1));
-          rsb2[u & 1] = fadd2(rsb2[u & 1], f2(__uint_as_float(pk[u] << 16), __uint_as_float(pk[u] & 0xffff0000u)));
-        }
-        tmem_st16(tS + ch * 16, pk);
-      }
-      {
-        float a0, a1, b0, b1;
-        f2_split(fadd2(rs2[0], rs2[1]), a0, a1);
-        f2_split(fadd2(rsb2[0], rsb2[1]), b0, b1);
-        l += a0 + a1;
-        lb += b0 + b1;
-      }
+      if (full)
+        exp_row_to_tmem<true>(s, sl2, ms, tS, l, lb);
+      else
+        exp_row_to_tmem<false>(s, sl2, ms, tS, l, lb);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
