@@ -24,9 +24,13 @@
 //   warps 4-7   the same for query columns 64-127
 //   warps 8-11  dQ drain (one thread per query row of the dQ tile) and the
 //               final dK/dV epilogue (one thread per key row)
-//   warp 12     tcgen05.mma issuer and TMEM owner
+//   warp 12     tcgen05.mma issuer, stream A (S^T, dV) and TMEM owner
 //   warp 13     TMA producer (tiles of Q and dO, and the tile's LSE / D rows)
-//   warps 14-15 idle (they complete the fourth warpgroup)
+//   warp 14     tcgen05.mma issuer, stream B (dP^T, dK, dQ)
+//   warp 15     idle (completes the fourth warpgroup)
+// The two MMA streams touch disjoint TMEM regions (A: S^T and dV; B: dP^T, dK
+// and dQ), so each keeps its own order and a thread blocked pushing one
+// stream's instructions into a full tensor-core queue never delays the other.
 // Registers: 128 per thread at launch; the fourth warpgroup gives up 56 and
 // the drain takes them (128 + 128 + 184 + 72 = 4 * 128), so a drain thread
 // holds a whole dQ row and releases the TMEM tile before its reductions.
@@ -185,6 +189,29 @@ __device__ __forceinline__ void stage_row32_bf16(uint8_t* tile, int r, int c, co
   }
 }
 
+// P^T = 2^(S^T * scale_log2 - LSE_q * log2 e) for one key row and 64 query
+// columns (LSE values broadcast from shared memory, 16 bytes per load).
+// kPoly: one pair in four on the FMA pipe (exp2_poly2), unmasked tiles only.
+template <bool kPoly>
+__device__ __forceinline__ void exp_cols64(const uint32_t (&sv)[64], const float* Lv, float sl2, float (&pv)[64]) {
+#pragma unroll
+  for (int c4 = 0; c4 < 16; ++c4) {
+    const float4 l4 = reinterpret_cast<const float4*>(Lv)[c4];
+    const float x0 = fmaf(__uint_as_float(sv[4 * c4 + 0]), sl2, -l4.x);
+    const float x1 = fmaf(__uint_as_float(sv[4 * c4 + 1]), sl2, -l4.y);
+    const float x2 = fmaf(__uint_as_float(sv[4 * c4 + 2]), sl2, -l4.z);
+    const float x3 = fmaf(__uint_as_float(sv[4 * c4 + 3]), sl2, -l4.w);
+    pv[4 * c4 + 0] = fast_exp2(x0);
+    pv[4 * c4 + 1] = fast_exp2(x1);
+    if (kPoly && (c4 & 1)) {
+      exp2_poly2(x2, x3, pv[4 * c4 + 2], pv[4 * c4 + 3]);
+    } else {
+      pv[4 * c4 + 2] = fast_exp2(x2);
+      pv[4 * c4 + 3] = fast_exp2(x3);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- main kernel
 template <int D>
 __global__ void __launch_bounds__(512, 1)
@@ -248,7 +275,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(kv_full, 1);
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
+      mbar_init(&q_empty[i], 2);  // one commit from each MMA stream
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -256,7 +283,7 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
-    mbar_init(kv_done, 1);
+    mbar_init(kv_done, 2);  // dV (stream A) and dK (stream B) complete
     mbar_init(epi_bar, 128);
     *abort_flag = 0;
     fence_mbar_init();
@@ -309,8 +336,8 @@ __global__ void __launch_bounds__(512, 1)
           while (!mbar_try_wait(smem_u32(&q_full[s]), (issued[s] - 1) & 1) &&
                  globaltimer_ns() - t0 < kWaitLimitNs) {
           }
-    } else if (warp == 12 && lane == 0) {
-      // ---------------------------------------------------------- MMA issuer
+    } else if ((warp == 12 || warp == 14) && lane == 0) {
+      // ---------------------------------------------------------- MMA issuers
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aSt = smem_u32(sStage), aDS = smem_u32(sDS);
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, false, true);     // dV, dK (A from TMEM)
@@ -333,48 +360,63 @@ __global__ void __launch_bounds__(512, 1)
                   sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&q_full[0], 0, abort_flag);
-      if (ok) {
-        tc_fence_after();
-        kmajor_nt(C::kColS, aK, st_q(0));
-        umma_commit(s_full);
-        kmajor_nt(C::kColDP, aV, st_do(0));
-        umma_commit(dp_full);
-      }
-      for (int it = 0; ok && it < total; ++it) {
-        const int s = it % C::kStages;
-        const int s1 = (it + 1) % C::kStages;
-        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
-        tc_fence_after();
-        ts_acc(C::kColDV, C::kColS, st_do(s), it > 0);  // dV += P^T dO
-        if (it + 1 < total) {
-          if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+      if (warp == 12) {
+        // stream A: S^T_i = K Q_i^T, then dV += P_i^T dO_i once P_i is in TMEM
+        if (ok) {
           tc_fence_after();
-          kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
+          kmajor_nt(C::kColS, aK, st_q(0));
           umma_commit(s_full);
         }
-        if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
-        tc_fence_after();
-        ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
-        if (!C::kAliasDq && it > 0) {
-          if (!(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag))) break;
+        for (int it = 0; ok && it < total; ++it) {
+          const int s = it % C::kStages;
+          const int s1 = (it + 1) % C::kStages;
+          if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
           tc_fence_after();
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k)  // dQ_i = dS K (both operands MN-major in smem)
-          umma_ss(tmem + C::kColDQ, sdesc_sw128(aDS + k * 2048, 16384, 1024),
-                  sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
-        umma_commit(dq_full);
-        umma_commit(&q_empty[s]);
-        if (it + 1 < total) {
-          if (C::kAliasDq) {
-            if (!(ok = mbar_wait(dq_empty, it & 1, abort_flag))) break;
+          ts_acc(C::kColDV, C::kColS, st_do(s), it > 0);  // dV += P^T dO
+          umma_commit(&q_empty[s]);
+          if (it + 1 < total) {
+            if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kStages) & 1, abort_flag))) break;
             tc_fence_after();
+            kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
+            umma_commit(s_full);
           }
-          kmajor_nt(C::kColDP, aV, st_do(s1));  // dP^T of the next query tile
+        }
+        if (ok) umma_commit(kv_done);
+      } else {
+        // stream B: dP^T_i = V dO_i^T; once dS_i is ready dK += dS_i^T Q_i and dQ_i = dS_i K
+        if (ok) {
+          tc_fence_after();
+          kmajor_nt(C::kColDP, aV, st_do(0));
           umma_commit(dp_full);
         }
+        for (int it = 0; ok && it < total; ++it) {
+          const int s = it % C::kStages;
+          const int s1 = (it + 1) % C::kStages;
+          if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
+          tc_fence_after();
+          ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
+          if (!C::kAliasDq && it > 0) {
+            if (!(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)  // dQ_i = dS K (both operands MN-major in smem)
+            umma_ss(tmem + C::kColDQ, sdesc_sw128(aDS + k * 2048, 16384, 1024),
+                    sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
+          umma_commit(dq_full);
+          umma_commit(&q_empty[s]);
+          if (it + 1 < total) {
+            if (C::kAliasDq) {
+              if (!(ok = mbar_wait(dq_empty, it & 1, abort_flag))) break;
+            }
+            if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+            tc_fence_after();
+            kmajor_nt(C::kColDP, aV, st_do(s1));  // dP^T of the next query tile
+            umma_commit(dp_full);
+          }
+        }
+        if (ok) umma_commit(kv_done);
       }
-      if (ok) umma_commit(kv_done);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -405,11 +447,10 @@ __global__ void __launch_bounds__(512, 1)
       tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
       tmem_wait_ld();
       float pv[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float lv = Lv[c];
-        pv[c] = fast_exp2(fmaf(__uint_as_float(sv[c]), sl2, -lv));
-      }
+      if (full)
+        exp_cols64<true>(sv, Lv, sl2, pv);
+      else
+        exp_cols64<false>(sv, Lv, sl2, pv);
       if (!full) {  // tiles on the diagonal / window edge only: one branch, not one per element
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -437,11 +478,17 @@ __global__ void __launch_bounds__(512, 1)
         tmem_wait_ld();
         uint32_t ds[16];
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const uint32_t pp = pk[h * 16 + u];
-          const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
-          const float d0 = Dv[32 * h + 2 * u], d1 = Dv[32 * h + 2 * u + 1];
-          ds[u] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * u]) - d0), p1 * (__uint_as_float(dv[2 * u + 1]) - d1));
+        for (int u2 = 0; u2 < 8; ++u2) {
+          const float4 d4 = reinterpret_cast<const float4*>(Dv)[8 * h + u2];
+          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int u = 2 * u2 + e;
+            const uint32_t pp = pk[h * 16 + u];
+            const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
+            ds[u] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * u]) - dd[2 * e]),
+                                p1 * (__uint_as_float(dv[2 * u + 1]) - dd[2 * e + 1]));
+          }
         }
         // dS^T (packed) over dP^T columns this thread has already read; dS into
         // shared memory as rows = keys, columns = queries (MN-major A of dQ).

@@ -261,6 +261,27 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 2^x for a pair of values on the FMA pipe.  Cody-Waite reduction x = n + f,
+// n = rint(x) (added to the exponent field), f in [-1/2, 1/2], and the degree-3
+// polynomial with minimal maximum relative error for 2^f on that interval
+// (7.5e-5; coefficients from exp2_poly.py, a Remez exchange).  x is clamped at
+// -126 so the exponent add cannot wrap; callers use it on unmasked tiles only.
+__device__ __forceinline__ void exp2_poly2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: adding it rounds to an integer
+  const uint64_t xx = f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t t = fadd2(xx, f2(kMagic, kMagic));
+  const uint64_t n = fadd2(t, f2(-kMagic, -kMagic));
+  const uint64_t f = ffma2(n, f2(-1.f, -1.f), xx);
+  uint64_t p = ffma2(f, f2(0.05517167f, 0.05517167f), f2(0.24261113f, 0.24261113f));
+  p = ffma2(p, f, f2(0.69326097f, 0.69326097f));
+  p = ffma2(p, f, f2(0.99992806f, 0.99992806f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

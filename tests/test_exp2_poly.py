@@ -10,7 +10,7 @@ import numpy as np
 from exact_io_aware_online_b200 import exp2_poly as E
 
 KERNEL = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                      "exact_io_aware_online_b200", "csrc", "fwd_sm100.cuh")
+                      "exact_io_aware_online_b200", "csrc", "sm100_ptx.cuh")
 
 
 def _kernel_coefficients():
