@@ -36,8 +36,14 @@ What it computes, and where each step is stated:
 * GQA -- query head h reads kv head h // (H / Hkv); the gradients of a kv
   head sum over its query heads.  The guide page only names grouped-query
   attention, so this contiguous grouping is a reading.
-* Fully masked rows (impossible in the shipped workloads, where the diagonal
-  is always allowed) give O = 0, LSE = -inf and zero gradients.
+* Block-sparse attention -- "FlashAttention paper" page, section "What it does
+  not claim": block sparsity is a separate extension of the same algorithm.
+  Reading: a 0/1 mask M over 128 x 128 blocks of the score matrix (per head or
+  shared), and a key is allowed only if the causal / window predicate holds
+  AND M[i // 128][j // 128] = 1.
+* Fully masked rows (impossible in the shipped dense workloads, where the
+  diagonal is always allowed; possible under a block mask) give O = 0,
+  LSE = -inf and zero gradients.
 
 Implementation notes, none of which changes a value: rows are processed in
 blocks (each row's softmax is still computed over its whole key range at once),
@@ -51,10 +57,14 @@ import numpy as np
 __all__ = ["allowed", "attention_probs", "forward", "backward", "row_dot"]
 
 
-def allowed(rows: np.ndarray, cols: np.ndarray, causal: bool, window: int) -> np.ndarray:
+BLOCK = 128  # block size of block-sparse masks (rows and columns)
+
+
+def allowed(rows: np.ndarray, cols: np.ndarray, causal: bool, window: int, block_mask=None) -> np.ndarray:
     """Boolean mask a[i, j]: may query ``rows[i]`` attend to key ``cols[j]``?
 
-    causal -> j <= i; window >= 0 -> |i - j| <= window; window = -1 -> no band.
+    causal -> j <= i; window >= 0 -> |i - j| <= window; window = -1 -> no band;
+    block_mask (2-D 0/1 array over 128 x 128 blocks) -> block (i//128, j//128) on.
     """
     r = np.asarray(rows)[:, None]
     c = np.asarray(cols)[None, :]
@@ -63,6 +73,9 @@ def allowed(rows: np.ndarray, cols: np.ndarray, causal: bool, window: int) -> np
         ok &= c <= r
     if window >= 0:
         ok &= np.abs(r - c) <= window
+    if block_mask is not None:
+        bm = np.asarray(block_mask).astype(bool)
+        ok &= bm[(r // BLOCK), (c // BLOCK)]
     return ok
 
 
@@ -76,21 +89,21 @@ def _key_range(r0: int, r1: int, n: int, causal: bool, window: int) -> tuple[int
     return lo, max(lo, hi)
 
 
-def _scores(q_rows, k_keys, scale, rows, keys, causal, window):
+def _scores(q_rows, k_keys, scale, rows, keys, causal, window, block_mask=None):
     s = scale * (q_rows @ k_keys.T)
-    ok = allowed(rows, keys, causal, window)
+    ok = allowed(rows, keys, causal, window, block_mask)
     s = np.where(ok, s, -np.inf)
     return s, ok
 
 
-def attention_probs(q_rows, k_keys, scale, rows, keys, causal, window):
+def attention_probs(q_rows, k_keys, scale, rows, keys, causal, window, block_mask=None):
     """Safe softmax of the masked, scaled scores of one head.
 
     Returns (P, m, l): P[i, j] probabilities, m the row max of the scaled
     scores, l = sum_j exp(S_ij - m_i).  Rows with no allowed key get P = 0,
     m = -inf, l = 0.
     """
-    s, ok = _scores(q_rows, k_keys, scale, rows, keys, causal, window)
+    s, ok = _scores(q_rows, k_keys, scale, rows, keys, causal, window, block_mask)
     m = s.max(axis=1) if s.shape[1] else np.full(s.shape[0], -np.inf)
     dead = ~np.isfinite(m)
     m_safe = np.where(dead, 0.0, m)
@@ -114,12 +127,20 @@ def _heads(q, k):
     return b, h, hkv, n, d, h // hkv
 
 
+def _head_mask(block_mask, b, h):
+    if block_mask is None:
+        return None
+    bm = np.asarray(block_mask)
+    return bm if bm.ndim == 2 else bm[b, h]
+
+
 def forward(q, k, v, scale: float, causal: bool = False, window: int = -1,
-            heads=None, row_block: int = 2048):
+            heads=None, row_block: int = 2048, block_mask=None):
     """O [B,H,N,d] and LSE [B,H,N] in fp64.
 
     q: [B,H,N,d]; k, v: [B,Hkv,N,d].  ``heads`` optionally restricts the work to
-    a list of (b, h) pairs; other heads are left as NaN.
+    a list of (b, h) pairs; other heads are left as NaN.  ``block_mask``: 0/1
+    over 128 x 128 blocks, shape [nb, nb] (all heads) or [B, H, nb, nb].
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
     b_, h_, _, n, d, g = _heads(q, k)
@@ -133,7 +154,7 @@ def forward(q, k, v, scale: float, causal: bool = False, window: int = -1,
             lo, hi = _key_range(r0, r1, n, causal, window)
             rows, keys = np.arange(r0, r1), np.arange(lo, hi)
             p, m, l = attention_probs(q[b, h, r0:r1], k[b, kvh, lo:hi], scale,
-                                      rows, keys, causal, window)
+                                      rows, keys, causal, window, _head_mask(block_mask, b, h))
             o[b, h, r0:r1] = p @ v[b, kvh, lo:hi]
             with np.errstate(divide="ignore"):
                 lse[b, h, r0:r1] = np.where(l > 0, m + np.log(np.where(l > 0, l, 1.0)), -np.inf)
@@ -146,7 +167,7 @@ def row_dot(p: np.ndarray, dp: np.ndarray) -> np.ndarray:
 
 
 def backward(q, k, v, do, scale: float, causal: bool = False, window: int = -1,
-             heads=None, row_block: int = 2048):
+             heads=None, row_block: int = 2048, block_mask=None):
     """dQ [B,H,N,d], dK and dV [B,Hkv,N,d] of L = sum(dO * O), in fp64.
 
     S and P are recomputed from Q and K (no saved forward state is used).
@@ -167,7 +188,7 @@ def backward(q, k, v, do, scale: float, causal: bool = False, window: int = -1,
             rows, keys = np.arange(r0, r1), np.arange(lo, hi)
             kk, vv = k[b, kvh, lo:hi], v[b, kvh, lo:hi]
             qq, dd = q[b, h, r0:r1], do[b, h, r0:r1]
-            p, _, _ = attention_probs(qq, kk, scale, rows, keys, causal, window)
+            p, _, _ = attention_probs(qq, kk, scale, rows, keys, causal, window, _head_mask(block_mask, b, h))
             dv[b, kvh, lo:hi] += p.T @ dd
             dp = dd @ vv.T
             ds = p * (dp - row_dot(p, dp)[:, None])

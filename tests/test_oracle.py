@@ -304,3 +304,60 @@ def test_forward_agrees_with_torch_sdpa_at_fp32_workload_shape():
     np.testing.assert_allclose(dq, qr.grad.numpy(), atol=1e-11)
     np.testing.assert_allclose(dk, kr.grad.numpy(), atol=1e-11)
     np.testing.assert_allclose(dv, vr.grad.numpy(), atol=1e-11)
+
+
+# --------------------------------------------------------------------------
+# Block-sparse masks (128 x 128 blocks)
+# --------------------------------------------------------------------------
+def test_block_mask_all_ones_equals_dense():
+    n, d = 300, 8
+    q, k, v, do = (_rand((1, 2, n, d), s) for s in (100, 101, 102, 103))
+    nb = (n + 127) // 128
+    ones = np.ones((nb, nb), dtype=np.uint8)
+    for causal, window in MODES:
+        o1, l1 = ref.forward(q, k, v, 0.3, causal, window)
+        o2, l2 = ref.forward(q, k, v, 0.3, causal, window, block_mask=ones)
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(l1, l2)
+        g1 = ref.backward(q, k, v, do, 0.3, causal, window)
+        g2 = ref.backward(q, k, v, do, 0.3, causal, window, block_mask=ones)
+        for a, b in zip(g1, g2):
+            np.testing.assert_array_equal(a, b)
+
+
+def test_block_diagonal_mask_equals_independent_blocks():
+    """With only diagonal blocks on, each 128-row block is its own attention
+    problem: the result equals the dense oracle run on each block alone."""
+    n, d = 333, 6
+    q, k, v, do = (_rand((1, 1, n, d), s) for s in (110, 111, 112, 113))
+    nb = (n + 127) // 128
+    diag = np.eye(nb, dtype=np.uint8)
+    o, lse = ref.forward(q, k, v, 0.4, block_mask=diag)
+    dq, dk, dv = ref.backward(q, k, v, do, 0.4, block_mask=diag)
+    for bi in range(nb):
+        sl = slice(128 * bi, min(n, 128 * (bi + 1)))
+        ob, lb = ref.forward(q[:, :, sl], k[:, :, sl], v[:, :, sl], 0.4)
+        gq, gk, gv = ref.backward(q[:, :, sl], k[:, :, sl], v[:, :, sl], do[:, :, sl], 0.4)
+        np.testing.assert_allclose(o[:, :, sl], ob, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, sl], lb, atol=1e-13)
+        np.testing.assert_allclose(dq[:, :, sl], gq, atol=1e-13)
+        np.testing.assert_allclose(dk[:, :, sl], gk, atol=1e-13)
+        np.testing.assert_allclose(dv[:, :, sl], gv, atol=1e-13)
+
+
+def test_block_mask_fully_masked_rows_and_per_head_masks():
+    n, d = 260, 4
+    q, k, v, do = (_rand((1, 2, n, d), s) for s in (120, 121, 122, 123))
+    bm = np.zeros((1, 2, 3, 3), dtype=np.uint8)
+    bm[0, 0] = np.tril(np.ones((3, 3)))
+    bm[0, 1, 0, 0] = 1  # head 1: only block (0, 0); rows >= 128 see nothing
+    o, lse = ref.forward(q, k, v, 0.5, block_mask=bm)
+    assert np.all(o[0, 1, 128:] == 0) and np.all(lse[0, 1, 128:] == -np.inf)
+    dq, dk, dv = ref.backward(q, k, v, do, 0.5, block_mask=bm)
+    assert np.all(dq[0, 1, 128:] == 0)
+    o_dense, _ = ref.forward(q[:, 1:2, :128], k[:, 1:2, :128], v[:, 1:2, :128], 0.5)
+    np.testing.assert_allclose(o[0, 1, :128], o_dense[0, 0], atol=1e-13)
+    # head 0: block-causal mask = causal at block granularity, a superset of causal
+    o_c, _ = ref.forward(q[:, :1], k[:, :1], v[:, :1], 0.5, causal=True, block_mask=bm[:, :1])
+    o_cc, _ = ref.forward(q[:, :1], k[:, :1], v[:, :1], 0.5, causal=True)
+    np.testing.assert_allclose(o_c, o_cc, atol=1e-13)
