@@ -210,6 +210,7 @@ def config_of(w: W.Workload, world: int):
     in_bytes = (2 * w.B * w.H + 2 * w.B * w.Hkv) * w.N * w.d * (2 if w.dtype == "bf16" else 4)
     return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
             "window": w.window, "scale": "1/sqrt(d)", "parallelism": f"replicas{world}" if world > 1 else "single",
+            "fwd_splits": getattr(config_of, "splits", 0),
             "l2": f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of Q,K,V,dO per step per GPU (no flush)"}
 
 
@@ -235,6 +236,10 @@ def run_ours(args, w, world, rank, local):
     dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
     ws = torch.empty(fa.bwd_workspace_size(B, H, N, d, fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP32),
                      dtype=torch.uint8, device=dev)
+    ws_split = None
+    if args.splits:
+        ws_split = torch.empty(int(fa.lib().fa_fwd_splitkv_workspace_size(B, H, N, d, args.splits)),
+                               dtype=torch.uint8, device=dev)
     K = args.steps
     ev_f = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     ev_b = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -242,7 +247,11 @@ def run_ours(args, w, world, rank, local):
     def step(i=None):
         if i is not None:
             fa.set_timing_events(*ev_f[i])
-        fa.fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, out=o, lse=lse)
+        if args.splits:
+            fa.fwd_splitkv(x["q"], x["k"], x["v"], args.splits, w.scale, w.causal, w.window, out=o, lse=lse,
+                           workspace=ws_split)
+        else:
+            fa.fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, out=o, lse=lse)
         if i is not None:
             fa.set_timing_events(*ev_b[i])
         fa.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], w.scale, w.causal, w.window, workspace=ws,
@@ -379,11 +388,13 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--splits", type=int, default=0, help="split-KV forward with this many key chunks (0: off)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
     w = W.WORKLOADS[args.workload]
+    config_of.splits = args.splits
     try:
         if args.impl == "reference":
             return run_reference(args, w, world, rank)

@@ -14,7 +14,7 @@ import os
 import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
-           "exported_names", "set_timing_events", "bwd_noalloc", "LIB_PATH", "HEADER_PATH"]
+           "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -64,6 +64,10 @@ def lib() -> ctypes.CDLL:
     L.fa_set_timing_events.restype = None
     L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp]
     L.fa_bwd_noalloc.restype = i
+    L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, i, vp, sz, i, vp]
+    L.fa_fwd_splitkv.restype = i
+    L.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i]
+    L.fa_fwd_splitkv_workspace_size.restype = sz
     _lib = L
     return L
 
@@ -106,6 +110,25 @@ def fwd(q, k, v, scale: float | None = None, causal: bool = False, window: int =
                         B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
                         _stream_ptr(q.device))
     _check(code, "fa_fwd")
+    return o, l
+
+
+def fwd_splitkv(q, k, v, num_splits: int, scale: float | None = None, causal: bool = False, window: int = -1,
+                out=None, lse=None, workspace=None):
+    """fwd() with each query block's key range split into `num_splits` chunks
+    (partials merged on the device); bf16 only."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = int(lib().fa_fwd_splitkv_workspace_size(B, H, N, d, int(num_splits)))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    code = lib().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), int(num_splits),
+                                ws.data_ptr(), ws.numel(), _dtype_code(q), _stream_ptr(q.device))
+    _check(code, "fa_fwd_splitkv")
     return o, l
 
 

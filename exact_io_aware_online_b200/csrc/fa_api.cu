@@ -98,15 +98,25 @@ fa::SimtParams simt_params(int B, int H, int Hkv, int N, float scale, int causal
   return s;
 }
 
+inline size_t splitkv_ws_bytes(int B, int H, int N, int d, int splits) {
+  const size_t nq2 = static_cast<size_t>((N + 255) / 256) * 256;
+  return align256(static_cast<size_t>(splits) * B * H * nq2 * d * 4) +
+         align256(static_cast<size_t>(splits) * B * H * nq2 * 16);
+}
+
+// splits == 0: the plain forward; splits >= 1: split-KV partials into `ws`
+// followed by the merge kernel.
 template <int D>
 fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
-                   float scale, int causal, int window, cudaStream_t st) {
+                   float scale, int causal, int window, cudaStream_t st, int splits = 0, void* ws = nullptr) {
   using C = fa::FwdCfg<D>;
   CUtensorMap tq, tk, tv, to;
   if (!make_tile_map(&tq, q, B * H, N, D) || !make_tile_map(&tk, k, B * Hkv, N, D) ||
       !make_tile_map(&tv, v, B * Hkv, N, D) || !make_tile_map(&to, o, B * H, N, D))
     return FA_ERR_CUDA;
-  if (!set_smem(fa::fwd_sm100_kernel<D>, C::kSmemBytes)) return FA_ERR_CUDA;
+  if (!set_smem(fa::fwd_sm100_kernel<D, false>, C::kSmemBytes) ||
+      !set_smem(fa::fwd_sm100_kernel<D, true>, C::kSmemBytes))
+    return FA_ERR_CUDA;
   fa::FwdParams p{};
   p.lse = lse;
   p.B = B;
@@ -126,9 +136,23 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
     p.group = std::min(p.group, B * H);
   }
   const unsigned grid = static_cast<unsigned>(p.npairs) * B * H;
+  if (splits == 0) {
+    mark_start(st);
+    fa::fwd_sm100_kernel<D, false><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    mark_stop(st);
+    return launched();
+  }
+  p.splits = splits;
+  p.nq2 = p.npairs * 256;
+  p.part_o = static_cast<float*>(ws);
+  p.part_m = reinterpret_cast<float4*>(static_cast<uint8_t*>(ws) +
+                                       align256(static_cast<size_t>(splits) * B * H * p.nq2 * D * 4));
   mark_start(st);
-  fa::fwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+  fa::fwd_sm100_kernel<D, true><<<grid * splits, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
   mark_stop(st);
+  if (launched() != FA_OK) return FA_ERR_CUDA;
+  const unsigned cgrid = static_cast<unsigned>(B * H) * ((N + 31) / 32);
+  fa::fwd_combine_kernel<D><<<cgrid, 256, 0, st>>>(p, o);
   return launched();
 }
 
@@ -282,6 +306,28 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                    : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st);
   return d == 64 ? fwd_f32<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st)
                  : fwd_f32<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st);
+}
+
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits) {
+  if (check_common(B, H, 1, N, d, 1.0f, -1, FA_BF16) != FA_OK) return 0;
+  if (num_splits < 1 || num_splits > fa::kMaxSplits) return 0;
+  return splitkv_ws_bytes(B, H, N, d, num_splits);
+}
+
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                         int N, int d, float scale, int causal, int window, int num_splits, void* workspace,
+                         size_t ws_bytes, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (num_splits < 1 || num_splits > fa::kMaxSplits) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < splitkv_ws_bytes(B, H, N, d, num_splits)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, num_splits, workspace)
+                 : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, num_splits, workspace);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype) {

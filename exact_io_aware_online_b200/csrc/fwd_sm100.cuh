@@ -41,7 +41,21 @@ struct FwdParams {
   int npairs;     // ceil(N / 256): query-tile pairs per head
   int ntiles_kv;  // ceil(N / 128)
   int group;      // heads per rasterisation group (kept L2-resident together)
+  // split-KV mode only: each CTA covers one of `splits` contiguous chunks of its
+  // key-tile range and writes partial results instead of O and the logsumexp.
+  int splits;
+  int nq2;         // npairs * 256: rows per head in the partial buffers
+  float* part_o;   // [splits][B*H][nq2][D] fp32 unnormalised O~, lane-interleaved (fwd_part_index)
+  float4* part_m;  // [splits][B*H][nq2] {m (log2 units), l, l_bf16, 0}
 };
+
+// Partial-output layout: row n = 32 g + lane; the 16-byte unit u (columns
+// 4u..4u+3) of 32 consecutive rows is contiguous, so a warp whose lane owns a
+// row stores and loads 512 contiguous bytes per unit.
+template <int D>
+__device__ __forceinline__ size_t fwd_part_unit(size_t split_bh, int nq2, int g, int u) {
+  return ((split_bh * static_cast<size_t>(nq2 / 32) + g) * (D / 4) + u) * 128;
+}
 
 template <int D>
 struct FwdCfg {
@@ -99,7 +113,7 @@ __device__ __forceinline__ void exp_row_to_tmem(const float (&s)[128], float sl2
   lb += b0 + b1;
 }
 
-template <int D>
+template <int D, bool kSplit>
 __global__ void __launch_bounds__(384, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -127,11 +141,13 @@ __global__ void __launch_bounds__(384, 1)
   // run together (their K/V stay in L2); inside a group the heaviest (last)
   // pairs under a causal mask go first.
   const int BH = p.B * p.H;
+  const int split = kSplit ? static_cast<int>(blockIdx.x) % p.splits : 0;
+  const int unit = kSplit ? static_cast<int>(blockIdx.x) / p.splits : static_cast<int>(blockIdx.x);
   const int per_group = p.group * p.npairs;
-  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int grp = unit / per_group;
   const int g0 = grp * p.group;
   const int gsz = min(p.group, BH - g0);
-  const int rem = static_cast<int>(blockIdx.x) - grp * per_group;
+  const int rem = unit - grp * per_group;
   const int pair = p.npairs - 1 - rem / gsz;
   const int bh = g0 + rem % gsz;
   const int b = bh / p.H, h = bh % p.H;
@@ -143,6 +159,11 @@ __global__ void __launch_bounds__(384, 1)
   if (p.window >= 0) {
     jlo = max(0, q0 - p.window) / 128;
     jhi = min(jhi, (qlast + p.window) / 128);
+  }
+  if (kSplit) {  // my contiguous chunk of the key-tile range (possibly empty)
+    const int chunk = (jhi - jlo + p.splits) / p.splits;
+    jlo += split * chunk;
+    jhi = min(jhi, jlo + chunk - 1);
   }
   const int nkv = jhi - jlo + 1;
 
@@ -177,10 +198,12 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(&tmQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128, bh);
+      if (nkv > 0) {
+        mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(&tmQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128, bh);
+      }
       int issued[C::kStages];
 #pragma unroll
       for (int i = 0; i < C::kStages; ++i) issued[i] = 0;
@@ -199,7 +222,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       // Never leave the CTA with copies still landing in shared memory.
       const unsigned long long t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(q_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      while (nkv > 0 && !mbar_try_wait(smem_u32(q_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
       }
       for (int s = 0; s < C::kStages; ++s)
         if (issued[s] > 0)
@@ -225,7 +248,7 @@ __global__ void __launch_bounds__(384, 1)
           umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8,
                   sdesc_sw128(aKV + slot * C::kTileBytes + k * 2048, 16384, 1024), kIdescO, acc || k > 0);
       };
-      bool ok = mbar_wait(q_full, 0, abort_flag);
+      bool ok = nkv > 0 && mbar_wait(q_full, 0, abort_flag);
       int it = 0;
       for (int jj = 0; ok && jj < nkv; ++jj, it += 2) {
         const int sK = it % C::kStages;
@@ -343,6 +366,27 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_before();
       mbar_arrive(&p_full[t]);
     }
+    if (kSplit) {
+      // ------------------------------------------------ partial results
+      const int n = tq0 + r;  // < nq2 always
+      const size_t sbh = static_cast<size_t>(split) * BH + bh;
+      if (nkv <= 0) {
+        p.part_m[sbh * p.nq2 + n] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
+      } else if (ok && (ok = mbar_wait(&o_full[t], 0, abort_flag))) {
+        tc_fence_after();
+        float* dst = p.part_o + fwd_part_unit<D>(sbh, p.nq2, n >> 5, 0) + 4 * lane;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(dst + 32 * (c + 4 * u)) = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+        }
+        p.part_m[sbh * p.nq2 + n] = make_float4(m_used, l, lb, 0.f);
+      }
+    } else {
     if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag);
     if (ok) {
       tc_fence_after();
@@ -377,12 +421,79 @@ __global__ void __launch_bounds__(384, 1)
       bulk_commit();
       bulk_wait_read0();
     }
+    }  // !kSplit
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- split-KV merge
+// Merges the per-chunk partial states of each query row with the block-merge
+// identity of "Flash attention and efficient attention" (Derivation, Step 3),
+// in base 2: m = max_s m_s, w_s = 2^(m_s - m),
+//   O = sum_s w_s O~_s / sum_s w_s lb_s,   LSE = (m + log2 sum_s w_s l_s) ln 2.
+// One block per (head, 32-row group): 32 threads compute the per-row weights,
+// all threads combine the 16-byte units (coalesced over rows), and the bf16
+// rows are written coalesced after a transpose through shared memory.
+constexpr int kMaxSplits = 16;
+
+template <int D>
+__global__ void __launch_bounds__(256) fwd_combine_kernel(const FwdParams p, void* out) {
+  __shared__ float wgt[32][kMaxSplits];
+  __shared__ float tile[32][D + 4];
+  const int groups = (p.N + 31) / 32;
+  const int BH = p.B * p.H;
+  const size_t bh = blockIdx.x / groups;
+  const int g = static_cast<int>(blockIdx.x % groups);
+  if (threadIdx.x < 32) {
+    const int n = 32 * g + threadIdx.x;
+    float m = -INFINITY;
+    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, p.part_m[(static_cast<size_t>(s) * BH + bh) * p.nq2 + n].x);
+    float wl = 0.f, wlb = 0.f;
+    for (int s = 0; s < p.splits; ++s) {
+      const float4 st = p.part_m[(static_cast<size_t>(s) * BH + bh) * p.nq2 + n];
+      const float w = (st.x == -INFINITY) ? 0.f : exp2f(st.x - m);
+      wgt[threadIdx.x][s] = w;
+      wl += w * st.y;
+      wlb += w * st.z;
+    }
+    const float inv = wlb > 0.f ? 1.f / wlb : 0.f;
+    for (int s = 0; s < p.splits; ++s) wgt[threadIdx.x][s] *= inv;
+    if (n < p.N) p.lse[bh * p.N + n] = (wl > 0.f) ? (m + log2f(wl)) * kLn2 : -INFINITY;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) {  // 32 rows x D/4 units, 256 threads
+    const int f = threadIdx.x + 256 * k;
+    const int u = f >> 5, l = f & 31;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < p.splits; ++s) {
+      const float w = wgt[l][s];
+      if (w == 0.f) continue;  // empty chunk or no allowed key: O~ unused
+      const float4 a = *reinterpret_cast<const float4*>(
+          p.part_o + fwd_part_unit<D>(static_cast<size_t>(s) * BH + bh, p.nq2, g, u) + 4 * l);
+      acc.x = fmaf(w, a.x, acc.x);
+      acc.y = fmaf(w, a.y, acc.y);
+      acc.z = fmaf(w, a.z, acc.z);
+      acc.w = fmaf(w, a.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(&tile[l][4 * u]) = acc;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < D / 32; ++k) {
+    const int f = threadIdx.x + 256 * k;
+    const int rr = f / (D / 4), u = f % (D / 4);
+    const int n = 32 * g + rr;
+    if (n >= p.N) continue;
+    uint2 v;
+    v.x = pack_bf16x2(tile[rr][4 * u + 0], tile[rr][4 * u + 1]);
+    v.y = pack_bf16x2(tile[rr][4 * u + 2], tile[rr][4 * u + 3]);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(out) + (bh * p.N + n) * D + 4 * u) = v;
   }
 }
 

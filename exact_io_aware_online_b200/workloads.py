@@ -53,6 +53,9 @@ WORKLOADS = {
                                                    16384, 128, "bf16", True, -1, 3, 0.01),
     "bf16_window128_h16_n32768_d64": Workload("bf16_window128_h16_n32768_d64", 1, 16, 16, 32768, 64,
                                               "bf16", False, 128, 4),
+    # not one of the stated workloads: a small-batch long-sequence case (too few
+    # query blocks to fill the GPU) used to measure the split-KV forward
+    "bf16_causal_b1h2_n16384_d128": Workload("bf16_causal_b1h2_n16384_d128", 1, 2, 2, 16384, 128, "bf16", True, -1, 5),
 }
 HEADLINE = "bf16_causal_b2h16_n8192_d128"
 

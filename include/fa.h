@@ -73,6 +73,28 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  fa_dtype dtype, void* stream);
 
 /*
+ * Split-KV forward: the same result as fa_fwd (o, lse), computed with the key
+ * range of every 256-row query block cut into num_splits contiguous chunks that
+ * run as separate CTAs.  Each chunk leaves its partial online-softmax state --
+ * running maximum m, sums l (and l of the bf16-rounded weights), unnormalised
+ * accumulator O~ -- in `workspace`; a second kernel merges them with the
+ * block-merge identity of "Flash attention and efficient attention",
+ * "Derivation: Incremental Softmax", Step 3 ("This generalizes to any number of
+ * blocks").  More CTAs for the same work: for small B*H with long N.
+ * bf16 only (FA_ERR_UNSUPPORTED for FA_FP32); 1 <= num_splits <= 16
+ * (FA_ERR_INVALID_ARG otherwise); workspace: caller-owned device memory of at
+ * least fa_fwd_splitkv_workspace_size() bytes, 16-byte aligned, contents
+ * irrelevant on entry.  Results are not bitwise equal to fa_fwd's (different
+ * summation order) and are deterministic.
+ */
+fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                         int N, int d, float scale, int causal, int window, int num_splits, void* workspace,
+                         size_t ws_bytes, fa_dtype dtype, void* stream);
+
+/* Workspace bytes fa_fwd_splitkv needs (0 for sizes it would reject). */
+size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes (fp32 row terms
  * D_i = sum_k dO_ik O_ik, prescaled LSE, and for bf16 a float dQ accumulator).
  * Returns 0 for sizes fa_bwd would reject.

@@ -21,7 +21,7 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version", "fa_set_timing_events"):
+              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size"):
         assert n in names
 
 
@@ -103,3 +103,32 @@ def test_python_helpers_fail_loudly_without_cuda():
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(Exception):
         fa.fwd(q, q, q)
+
+
+def _split(L, ws=A, ws_bytes=None, **kw):
+    a = dict(B=1, H=2, Hkv=1, N=300, d=128, scale=0.088, causal=1, window=-1, splits=3, dtype=0)
+    a.update(kw)
+    if ws_bytes is None:
+        ws_bytes = L.fa_fwd_splitkv_workspace_size(a["B"], a["H"], a["N"], a["d"], max(1, min(16, a["splits"])))
+    ptrs = [kw.get(n, A) for n in ("q", "k", "v", "o", "lse")]
+    return L.fa_fwd_splitkv(*ptrs, a["B"], a["H"], a["Hkv"], a["N"], a["d"], ctypes.c_float(a["scale"]),
+                            a["causal"], a["window"], a["splits"], ws, ws_bytes, a["dtype"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(lse=None), 1), (dict(splits=0), 1), (dict(splits=17), 1), (dict(H=3, Hkv=2), 1),
+    (dict(dtype=1), 2), (dict(d=96), 2), (dict(ws=None), 4), (dict(ws_bytes=100), 4), (dict(ws=A + 8), 3),
+    (dict(o=A + 4), 3),
+])
+def test_splitkv_rejects_bad_arguments(L, kw, code):
+    assert _split(L, **kw) == code
+
+
+@pytest.mark.parametrize("B,H,N,d,S", [(1, 1, 1, 64, 1), (2, 16, 8192, 128, 4), (1, 3, 300, 64, 16)])
+def test_splitkv_workspace_closed_form(L, B, H, N, d, S):
+    def a256(x):
+        return (x + 255) // 256 * 256
+    nq2 = (N + 255) // 256 * 256
+    assert L.fa_fwd_splitkv_workspace_size(B, H, N, d, S) == a256(S * B * H * nq2 * d * 4) + a256(S * B * H * nq2 * 16)
+    assert L.fa_fwd_splitkv_workspace_size(B, H, N, d, 0) == 0
+    assert L.fa_fwd_splitkv_workspace_size(B, H, N, d, 17) == 0
