@@ -211,6 +211,7 @@ def config_of(w: W.Workload, world: int):
     return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
             "window": w.window, "scale": "1/sqrt(d)", "parallelism": f"replicas{world}" if world > 1 else "single",
             "fwd_splits": getattr(config_of, "splits", 0),
+            "block_density": getattr(config_of, "block_density", None),
             "l2": f"inputs larger than L2: {in_bytes / 2**20:.0f} MiB of Q,K,V,dO per step per GPU (no flush)"}
 
 
@@ -236,6 +237,13 @@ def run_ours(args, w, world, rank, local):
     dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
     ws = torch.empty(fa.bwd_workspace_size(B, H, N, d, fa.FA_BF16 if w.dtype == "bf16" else fa.FA_FP32),
                      dtype=torch.uint8, device=dev)
+    bmask = None
+    if args.block_density is not None:
+        if w.window >= 0:
+            raise SystemExit("--block-density: window workloads are not supported")
+        m = W.block_mask(w.N, args.block_density, w.seed + 77, w.causal)
+        bmask = torch.from_numpy(m).to(dev)
+        flops_override = 4.0 * w.d * W.block_pairs(w.N, m, w.causal) * w.B * w.H
     ws_split = None
     if args.splits:
         ws_split = torch.empty(int(fa.lib().fa_fwd_splitkv_workspace_size(B, H, N, d, args.splits)),
@@ -247,15 +255,21 @@ def run_ours(args, w, world, rank, local):
     def step(i=None):
         if i is not None:
             fa.set_timing_events(*ev_f[i])
-        if args.splits:
+        if bmask is not None:
+            fa.fwd_blocksparse(x["q"], x["k"], x["v"], bmask, w.scale, w.causal, w.window, out=o, lse=lse)
+        elif args.splits:
             fa.fwd_splitkv(x["q"], x["k"], x["v"], args.splits, w.scale, w.causal, w.window, out=o, lse=lse,
                            workspace=ws_split)
         else:
             fa.fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.window, out=o, lse=lse)
         if i is not None:
             fa.set_timing_events(*ev_b[i])
-        fa.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], w.scale, w.causal, w.window, workspace=ws,
-               grads=(dq, dk, dv))
+        if bmask is not None:
+            fa.bwd_blocksparse(x["q"], x["k"], x["v"], o, lse, x["do"], bmask, w.scale, w.causal, w.window,
+                               workspace=ws, grads=(dq, dk, dv))
+        else:
+            fa.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], w.scale, w.causal, w.window, workspace=ws,
+                   grads=(dq, dk, dv))
         if i is not None:
             fa.set_timing_events(None, None)
 
@@ -297,6 +311,8 @@ def run_ours(args, w, world, rank, local):
         ms = float(t.item())
 
     fwd_f, bwd_f = W.flops(w)
+    if bmask is not None:  # the kept (query, key) pairs inside the switched-on blocks
+        fwd_f, bwd_f = flops_override, 2.5 * flops_override
     ms_step = ms / K
     value = world * (fwd_f + bwd_f) / (ms_step * 1e-3) / 1e12
 
@@ -389,12 +405,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--splits", type=int, default=0, help="split-KV forward with this many key chunks (0: off)")
+    ap.add_argument("--block-density", type=float, default=None,
+                    help="block-sparse attention with a seeded mask keeping this fraction of 128x128 blocks")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
     w = W.WORKLOADS[args.workload]
     config_of.splits = args.splits
+    config_of.block_density = args.block_density
     try:
         if args.impl == "reference":
             return run_reference(args, w, world, rank)

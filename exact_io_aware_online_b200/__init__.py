@@ -14,7 +14,7 @@ import os
 import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
-           "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "LIB_PATH", "HEADER_PATH"]
+           "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -68,6 +68,11 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_splitkv.restype = i
     L.fa_fwd_splitkv_workspace_size.argtypes = [i, i, i, i, i]
     L.fa_fwd_splitkv_workspace_size.restype = sz
+    ll = ctypes.c_longlong
+    L.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, ll, i, vp]
+    L.fa_fwd_blocksparse.restype = i
+    L.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, ll, i, vp]
+    L.fa_bwd_blocksparse.restype = i
     _lib = L
     return L
 
@@ -166,6 +171,57 @@ def bwd_noalloc(q, k, v, o, lse, do, scale: float | None = None, causal: bool = 
                                 B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
                                 _stream_ptr(q.device))
     _check(code, "fa_bwd_noalloc")
+    return dq, dk, dv
+
+
+def _mask_args(block_mask, B, H):
+    """(device pointer, head stride) for a uint8 block mask of shape [nb, nb]
+    (shared) or [B, H, nb, nb] (per query head)."""
+    import torch
+    if block_mask.dtype != torch.uint8 or not block_mask.is_contiguous():
+        raise TypeError("block_mask must be a contiguous torch.uint8 tensor")
+    nb = block_mask.shape[-1]
+    if block_mask.dim() == 2:
+        return block_mask.data_ptr(), 0
+    if tuple(block_mask.shape) != (B, H, nb, nb):
+        raise ValueError("block_mask must be [nb, nb] or [B, H, nb, nb]")
+    return block_mask.data_ptr(), nb * nb
+
+
+def fwd_blocksparse(q, k, v, block_mask, scale: float | None = None, causal: bool = False, window: int = -1,
+                    out=None, lse=None):
+    """fwd() restricted to the 128 x 128 blocks that `block_mask` switches on."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    mp, hs = _mask_args(block_mask, B, H)
+    code = lib().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                    B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), mp, hs,
+                                    _dtype_code(q), _stream_ptr(q.device))
+    _check(code, "fa_fwd_blocksparse")
+    return o, l
+
+
+def bwd_blocksparse(q, k, v, o, lse, do, block_mask, scale: float | None = None, causal: bool = False,
+                    window: int = -1, workspace=None, grads=None):
+    """bwd() of fwd_blocksparse()."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    code_t = _dtype_code(q)
+    need = bwd_workspace_size(B, H, N, d, code_t)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    mp, hs = _mask_args(block_mask, B, H)
+    code = lib().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                                    ws.numel(), B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), mp, hs,
+                                    code_t, _stream_ptr(q.device))
+    _check(code, "fa_bwd_blocksparse")
     return dq, dk, dv
 
 

@@ -67,6 +67,10 @@ struct BwdParams {
   int causal, window;
   int ntiles;  // Np / 128
   int group;   // kv heads per rasterisation group (kept L2-resident together)
+  // block-sparse mode (non-null bmask): 0/1 per 128 x 128 block, [query block]
+  // [key block] per query head, bmask_hs elements apart (0: shared by all heads)
+  const uint8_t* bmask;
+  long long bmask_hs;
 };
 
 template <int D>
@@ -266,10 +270,32 @@ __global__ void __launch_bounds__(512, 1)
     ilo = max(ilo, max(0, k0 - p.window) / 128);
     ihi = min(ihi, (k0 + 127 + p.window) / 128);
   }
-  const int nq = ihi - ilo + 1;
-  const int total = nq * p.g;
-  auto q_tile = [&](int it) { return ilo + it % nq; };
-  auto q_head = [&](int it) { return b * p.H + kh * p.g + it / nq; };
+  // Work list: (query head hq of the group, query tile i) pairs in increasing
+  // order, skipping blocks a block-sparse mask switches off.  Every role walks
+  // it with its own QCursor, so all roles see the same sequence.
+  const int bh0 = b * p.H + kh * p.g;
+  auto active = [&](int hq, int i) {
+    return !p.bmask || p.bmask[(bh0 + hq) * p.bmask_hs + static_cast<long long>(i) * p.ntiles + j] != 0;
+  };
+  struct QCursor {
+    int hq, i;
+  };
+  auto advance = [&](QCursor c) {  // next active pair strictly after c
+    do {
+      if (++c.i > ihi) {
+        c.i = ilo;
+        ++c.hq;
+      }
+    } while (c.hq < p.g && !active(c.hq, c.i));
+    return c;
+  };
+  auto first = [&]() {
+    QCursor c{0, ilo};
+    if (!active(0, ilo)) c = advance(c);
+    return c;
+  };
+  int total = 0;
+  for (QCursor c = first(); c.hq < p.g; c = advance(c)) ++total;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -313,11 +339,12 @@ __global__ void __launch_bounds__(512, 1)
       int issued[C::kStages];
 #pragma unroll
       for (int i = 0; i < C::kStages; ++i) issued[i] = 0;
-      for (int it = 0; it < total; ++it) {
+      QCursor cur = first();
+      for (int it = 0; it < total; ++it, cur = advance(cur)) {
         const int s = it % C::kStages;
         if (!mbar_wait(&q_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[s], 2 * C::kTileBytes + C::kVecBytes);
-        const int row0 = q_tile(it) * 128, bh = q_head(it);
+        const int row0 = cur.i * 128, bh = bh0 + cur.hq;
         uint8_t* st = sStage + s * 2 * C::kTileBytes;
         for (int c = 0; c < C::kChunks; ++c) {
           tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
@@ -359,10 +386,10 @@ __global__ void __launch_bounds__(512, 1)
           umma_ts(tmem + dcol, tmem + acol + (k >> 2) * 64 + (k & 3) * 8,
                   sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
       };
-      bool ok = mbar_wait(kv_full, 0, abort_flag) && mbar_wait(&q_full[0], 0, abort_flag);
+      bool ok = mbar_wait(kv_full, 0, abort_flag) && (total == 0 || mbar_wait(&q_full[0], 0, abort_flag));
       if (warp == 12) {
         // stream A: S^T_i = K Q_i^T, then dV += P_i^T dO_i once P_i is in TMEM
-        if (ok) {
+        if (ok && total > 0) {
           tc_fence_after();
           kmajor_nt(C::kColS, aK, st_q(0));
           umma_commit(s_full);
@@ -384,7 +411,7 @@ __global__ void __launch_bounds__(512, 1)
         if (ok) umma_commit(kv_done);
       } else {
         // stream B: dP^T_i = V dO_i^T; once dS_i is ready dK += dS_i^T Q_i and dQ_i = dS_i K
-        if (ok) {
+        if (ok && total > 0) {
           tc_fence_after();
           kmajor_nt(C::kColDP, aV, st_do(0));
           umma_commit(dp_full);
@@ -431,9 +458,10 @@ __global__ void __launch_bounds__(512, 1)
     const float sl2 = p.scale_log2;
     const int ds_chunk = w;  // 64-column (128-byte) block of the dS tile
     bool ok = true;
-    for (int it = 0; it < total; ++it) {
+    QCursor cur = first();
+    for (int it = 0; it < total; ++it, cur = advance(cur)) {
       const int s = it % C::kStages;
-      const int q0 = q_tile(it) * 128 + 64 * w;  // first query of my columns
+      const int q0 = cur.i * 128 + 64 * w;  // first query of my columns
       const float* Lv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes) + 64 * w;
       const float* Dv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes + 512) + 64 * w;
       bool full = true;  // every (query, key) pair of my 64 columns allowed?
@@ -512,11 +540,12 @@ __global__ void __launch_bounds__(512, 1)
     const int r = wl * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
     bool ok = true;
-    for (int it = 0; it < total; ++it) {
+    QCursor cur = first();
+    for (int it = 0; it < total; ++it, cur = advance(cur)) {
       if (!(ok = mbar_wait(dq_full, it & 1, abort_flag))) break;
       tc_fence_after();
-      // my row is 32 * (4 * q_tile + wl) + lane: group 4 * q_tile + wl, slot `lane`
-      float* dst = p.dqacc + dqacc_unit<D>(q_head(it), p.Np, 4 * q_tile(it) + wl, 0) + 4 * lane;
+      // my row is 32 * (4 * i + wl) + lane: group 4 * i + wl, slot `lane`
+      float* dst = p.dqacc + dqacc_unit<D>(bh0 + cur.hq, p.Np, 4 * cur.i + wl, 0) + 4 * lane;
       uint32_t v[D];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c)
@@ -534,11 +563,18 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_off + C::kColDV + c, v);
-        tmem_wait_ld();
+        if (total > 0) {
+          tmem_ld32(tmem + lane_off + C::kColDV + c, v);
+          tmem_wait_ld();
+        } else {  // no query block reaches this key tile (block mask): dV = dK = 0
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = 0u;
+        }
         stage_row32_bf16(sV, r, c, v, 1.f);
-        tmem_ld32(tmem + lane_off + C::kColDK + c, v);
-        tmem_wait_ld();
+        if (total > 0) {
+          tmem_ld32(tmem + lane_off + C::kColDK + c, v);
+          tmem_wait_ld();
+        }
         stage_row32_bf16(sK, r, c, v, p.scale);
       }
       fence_proxy_async_smem();

@@ -108,14 +108,16 @@ inline size_t splitkv_ws_bytes(int B, int H, int N, int d, int splits) {
 // followed by the merge kernel.
 template <int D>
 fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
-                   float scale, int causal, int window, cudaStream_t st, int splits = 0, void* ws = nullptr) {
+                   float scale, int causal, int window, cudaStream_t st, int splits = 0, void* ws = nullptr,
+                   const uint8_t* bmask = nullptr, long long bmask_hs = 0) {
   using C = fa::FwdCfg<D>;
   CUtensorMap tq, tk, tv, to;
   if (!make_tile_map(&tq, q, B * H, N, D) || !make_tile_map(&tk, k, B * Hkv, N, D) ||
       !make_tile_map(&tv, v, B * Hkv, N, D) || !make_tile_map(&to, o, B * H, N, D))
     return FA_ERR_CUDA;
-  if (!set_smem(fa::fwd_sm100_kernel<D, false>, C::kSmemBytes) ||
-      !set_smem(fa::fwd_sm100_kernel<D, true>, C::kSmemBytes))
+  if (!set_smem(fa::fwd_sm100_kernel<D, false, false>, C::kSmemBytes) ||
+      !set_smem(fa::fwd_sm100_kernel<D, true, false>, C::kSmemBytes) ||
+      !set_smem(fa::fwd_sm100_kernel<D, false, true>, C::kSmemBytes))
     return FA_ERR_CUDA;
   fa::FwdParams p{};
   p.lse = lse;
@@ -129,6 +131,9 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   p.window = window;
   p.npairs = (N + 255) / 256;
   p.ntiles_kv = (N + 127) / 128;
+  p.bmask = bmask;
+  p.bmask_hs = bmask_hs;
+  p.nbt = p.ntiles_kv;
   {  // heads per group: Q, O and the (shared) K, V of a group within ~64 MiB of L2
     const double unit = static_cast<double>(N) * D * (4.0 + 4.0 / p.g);
     p.group = std::min(B * H, static_cast<int>(std::max(1.0, std::floor((64.0 * 1024 * 1024) / unit))));
@@ -138,7 +143,10 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   const unsigned grid = static_cast<unsigned>(p.npairs) * B * H;
   if (splits == 0) {
     mark_start(st);
-    fa::fwd_sm100_kernel<D, false><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    if (bmask)
+      fa::fwd_sm100_kernel<D, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    else
+      fa::fwd_sm100_kernel<D, false, false><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
     mark_stop(st);
     return launched();
   }
@@ -148,7 +156,7 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   p.part_m = reinterpret_cast<float4*>(static_cast<uint8_t*>(ws) +
                                        align256(static_cast<size_t>(splits) * B * H * p.nq2 * D * 4));
   mark_start(st);
-  fa::fwd_sm100_kernel<D, true><<<grid * splits, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+  fa::fwd_sm100_kernel<D, true, false><<<grid * splits, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
   mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   const unsigned cgrid = static_cast<unsigned>(B * H) * ((N + 31) / 32);
@@ -158,8 +166,12 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
 
 template <int D>
 fa_status fwd_f32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
-                  float scale, int causal, int window, cudaStream_t st) {
+                  float scale, int causal, int window, cudaStream_t st, const uint8_t* bmask = nullptr,
+                  long long bmask_hs = 0) {
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
+  s.bmask = bmask;
+  s.bmask_hs = bmask_hs;
+  s.nbt = (N + 127) / 128;
   s.q = static_cast<const float*>(q);
   s.k = static_cast<const float*>(k);
   s.v = static_cast<const float*>(v);
@@ -193,7 +205,7 @@ WsLayout ws_layout(int B, int H, int N, int d, fa_dtype dtype) {
 template <int D>
 fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                    void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
-                   int window, cudaStream_t st) {
+                   int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0) {
   using C = fa::BwdCfg<D>;
   const WsLayout w = ws_layout(B, H, N, D, FA_BF16);
   uint8_t* wb = static_cast<uint8_t*>(ws);
@@ -216,6 +228,8 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   p.causal = causal ? 1 : 0;
   p.window = window;
   p.ntiles = p.Np / 128;
+  p.bmask = bmask;
+  p.bmask_hs = bmask_hs;
   // kv heads per rasterisation group: keep each group's Q, dO, K, V and dQ
   // accumulator (about N*d*(4 + 8g) bytes per kv head) within ~64 MiB of L2.
   {
@@ -244,8 +258,11 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
 template <int D>
 fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                   void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
-                  int window, cudaStream_t st) {
+                  int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0) {
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
+  s.bmask = bmask;
+  s.bmask_hs = bmask_hs;
+  s.nbt = (N + 127) / 128;
   s.q = static_cast<const float*>(q);
   s.k = static_cast<const float*>(k);
   s.v = static_cast<const float*>(v);
@@ -328,6 +345,51 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, num_splits, workspace)
                  : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, num_splits, workspace);
+}
+
+fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                             int Hkv, int N, int d, float scale, int causal, int window, const unsigned char* block_mask,
+                             long long mask_head_stride, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (mask_head_stride < 0) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16)
+    return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, block_mask,
+                                  mask_head_stride)
+                   : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, block_mask,
+                                   mask_head_stride);
+  return d == 64 ? fwd_f32<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, block_mask, mask_head_stride)
+                 : fwd_f32<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, block_mask, mask_head_stride);
+}
+
+fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                             int H, int Hkv, int N, int d, float scale, int causal, int window,
+                             const unsigned char* block_mask, long long mask_head_stride, fa_dtype dtype,
+                             void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !block_mask) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (mask_head_stride < 0) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < ws_layout(B, H, N, d, dtype).total) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const long long hs = mask_head_stride;
+  if (dtype == FA_BF16)
+    return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
+                                  block_mask, hs)
+                   : bwd_bf16<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window,
+                                   st, block_mask, hs);
+  return d == 64 ? bwd_f32<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
+                               block_mask, hs)
+                 : bwd_f32<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
+                                block_mask, hs);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype) {

@@ -45,6 +45,12 @@ struct FwdParams {
   // key-tile range and writes partial results instead of O and the logsumexp.
   int splits;
   int nq2;         // npairs * 256: rows per head in the partial buffers
+  // block-sparse mode (non-null bmask): 0/1 per 128 x 128 block of the score
+  // matrix, [query block][key block], nbt x nbt per query head at bmask_hs
+  // elements apart (0: one mask for all heads).
+  const uint8_t* bmask;
+  long long bmask_hs;
+  int nbt;
   float* part_o;   // [splits][B*H][nq2][D] fp32 unnormalised O~, lane-interleaved (fwd_part_index)
   float4* part_m;  // [splits][B*H][nq2] {m (log2 units), l, l_bf16, 0}
 };
@@ -113,7 +119,7 @@ __device__ __forceinline__ void exp_row_to_tmem(const float (&s)[128], float sl2
   lb += b0 + b1;
 }
 
-template <int D, bool kSplit>
+template <int D, bool kSplit, bool kMask>
 __global__ void __launch_bounds__(384, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -165,7 +171,24 @@ __global__ void __launch_bounds__(384, 1)
     jlo += split * chunk;
     jhi = min(jhi, jlo + chunk - 1);
   }
-  const int nkv = jhi - jlo + 1;
+  // Block-sparse: only key tiles whose block is on for either query tile are
+  // visited (every role walks the same increasing sequence, see next_kv).
+  // (kMask: the block-sparse variant; the dense kernels compile none of this.)
+  const long long brow0 = kMask ? bh * p.bmask_hs + static_cast<long long>(2 * pair) * p.nbt : 0;
+  const bool has_row1 = 2 * pair + 1 < p.nbt;
+  auto block_on = [&](int t, int j) {  // block (query tile 2 pair + t, key tile j) on?
+    return t == 0 ? p.bmask[brow0 + j] != 0 : (has_row1 && p.bmask[brow0 + p.nbt + j] != 0);
+  };
+  auto next_kv = [&](int j) {  // first visited key tile >= j (jhi + 1 if none)
+    if (kMask)
+      while (j <= jhi && !block_on(0, j) && !block_on(1, j)) ++j;
+    return j;
+  };
+  int nkv = jhi - jlo + 1;
+  if (kMask) {
+    nkv = 0;
+    for (int j = next_kv(jlo); j <= jhi; j = next_kv(j + 1)) ++nkv;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -208,8 +231,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int i = 0; i < C::kStages; ++i) issued[i] = 0;
       int it = 0;
-      for (int jj = 0; jj < nkv && !*abort_flag; ++jj) {
-        const int kv0 = (jlo + jj) * 128;
+      int jcur = next_kv(jlo);
+      for (int jj = 0; jj < nkv && !*abort_flag; ++jj, jcur = next_kv(jcur + 1)) {
+        const int kv0 = jcur * 128;
         for (int which = 0; which < 2; ++which, ++it) {
           const int s = it % C::kStages;
           if (!mbar_wait(&kv_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
@@ -300,8 +324,11 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY, l = 0.f, lb = 0.f;
     bool ok = true;
-    for (int jj = 0; jj < nkv; ++jj) {
-      const int kv0 = (jlo + jj) * 128;
+    int jcur = next_kv(jlo);
+    for (int jj = 0; jj < nkv; ++jj, jcur = next_kv(jcur + 1)) {
+      const int kv0 = jcur * 128;
+      // block switched off for this query tile: every score of the tile is masked
+      const bool block_off = kMask && !block_on(t, jcur);
       if (!(ok = mbar_wait(&s_full[t], jj & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t sraw[128];
@@ -311,14 +338,14 @@ __global__ void __launch_bounds__(384, 1)
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sraw[c]);
-      bool full = kv0 + 127 < p.N;
+      bool full = kv0 + 127 < p.N && !block_off;
       if (p.causal) full = full && (kv0 + 127 <= tq0);
       if (p.window >= 0) full = full && (tq0 + 127 - kv0 <= p.window) && (kv0 + 127 - tq0 <= p.window);
       if (!full) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const int key = kv0 + c;
-          bool keep = key < p.N;
+          bool keep = key < p.N && !block_off;
           if (p.causal) keep = keep && key <= qrow;
           if (p.window >= 0) keep = keep && abs(qrow - key) <= p.window;
           if (!keep) s[c] = -INFINITY;
@@ -387,7 +414,7 @@ __global__ void __launch_bounds__(384, 1)
         p.part_m[sbh * p.nq2 + n] = make_float4(m_used, l, lb, 0.f);
       }
     } else {
-    if (ok) ok = mbar_wait(&o_full[t], 0, abort_flag);
+    if (ok && nkv > 0) ok = mbar_wait(&o_full[t], 0, abort_flag);
     if (ok) {
       tc_fence_after();
       const float inv = (lb > 0.f) ? 1.f / lb : 0.f;
@@ -395,8 +422,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
-        tmem_ld32(tO + c, o);
-        tmem_wait_ld();
+        if (nkv > 0) {
+          tmem_ld32(tO + c, o);
+          tmem_wait_ld();
+        } else {  // no key tile at all (block mask): O = 0, LSE = -inf
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
         const int chunk = c >> 6, u0 = (c & 63) >> 3;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {

@@ -35,10 +35,19 @@ struct SimtParams {
   int B, H, Hkv, N, g;
   float scale;
   int causal, window;
+  const uint8_t* bmask;  // optional 0/1 mask per 128 x 128 block, [head][nbt][nbt]
+  long long bmask_hs;    // elements between heads' masks (0: shared)
+  int nbt;               // ceil(N / 128)
 };
 
 __device__ __forceinline__ bool keep_ij(int i, int j, int causal, int window) {
   return (!causal || j <= i) && (window < 0 || abs(i - j) <= window);
+}
+
+// keep_ij and, under a block mask, block (i / 128, j / 128) of query head bh on.
+__device__ __forceinline__ bool keep_ijb(const SimtParams& p, int bh, int i, int j) {
+  if (!keep_ij(i, j, p.causal, p.window)) return false;
+  return !p.bmask || p.bmask[bh * p.bmask_hs + static_cast<long long>(i >> 7) * p.nbt + (j >> 7)] != 0;
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -105,7 +114,7 @@ __global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
     if (!active) continue;
     for (int jj = 0; jj < cnt; ++jj) {
       const int j = kt + jj;
-      if (!keep_ij(i, j, p.causal, p.window)) continue;
+      if (!keep_ijb(p, bh, i, j)) continue;
       float s = 0.f;
 #pragma unroll
       for (int e = 0; e < E; ++e) s = fmaf(q[e], sK[jj][lane + 32 * e], s);
@@ -188,7 +197,7 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
       if (!active) continue;
       for (int ii = 0; ii < cnt; ++ii) {
         const int i = it + ii;
-        if (!keep_ij(i, j, p.causal, p.window)) continue;
+        if (!keep_ijb(p, bh, i, j)) continue;
         float s = 0.f, dp = 0.f;
 #pragma unroll
         for (int e = 0; e < E; ++e) {
@@ -253,7 +262,7 @@ __global__ void __launch_bounds__(256) bwd_dq_f32_kernel(const SimtParams p) {
     if (!active) continue;
     for (int jj = 0; jj < cnt; ++jj) {
       const int j = kt + jj;
-      if (!keep_ij(i, j, p.causal, p.window)) continue;
+      if (!keep_ijb(p, bh, i, j)) continue;
       float s = 0.f, dp = 0.f;
 #pragma unroll
       for (int e = 0; e < E; ++e) {

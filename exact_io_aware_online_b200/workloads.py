@@ -109,3 +109,34 @@ def flops(w: Workload) -> tuple[float, float]:
         pairs = float(allowed_pairs(w.N, w.causal, w.window))
     fwd = 4.0 * w.d * pairs * heads
     return fwd, 2.5 * fwd
+
+
+def block_mask(N: int, density: float, seed: int, causal: bool):
+    """Seeded 0/1 mask over 128 x 128 blocks ([nb, nb], uint8) for measuring
+    block-sparse attention: each block on with probability `density`; under a
+    causal mask the upper triangle is dropped and the diagonal kept on."""
+    import numpy as np
+    nb = (N + 127) // 128
+    m = (np.random.default_rng(seed).random((nb, nb)) < density).astype(np.uint8)
+    if causal:
+        m = np.tril(m)
+        np.fill_diagonal(m, 1)
+    return m
+
+
+def block_pairs(N: int, mask, causal: bool) -> int:
+    """(query, key) pairs a causal (or unmasked) attention keeps inside the
+    blocks `mask` switches on, for one head."""
+    nb = mask.shape[0]
+    total = 0
+    for i in range(nb):
+        ri = min(128, N - 128 * i)
+        for j in range(nb):
+            if not mask[i, j]:
+                continue
+            cj = min(128, N - 128 * j)
+            if not causal or j < i:
+                total += ri * cj if (not causal or j < i) else 0
+            elif j == i:
+                total += ri * (ri + 1) // 2
+    return total

@@ -95,6 +95,32 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits);
 
 /*
+ * Block-sparse forward and backward: as fa_fwd / fa_bwd with an extra 0/1 mask
+ * over 128 x 128 blocks of the score matrix; a key is allowed only if the
+ * causal / window predicate allows it AND its block is on.  Block sparsity is
+ * named on the "FlashAttention paper" page ("What it does not claim") as a
+ * separate extension of the same tiled algorithm; switched-off blocks are never
+ * loaded or multiplied.
+ *  block_mask        device pointer, unsigned char, nb x nb per query head
+ *                    (nb = ceil(N / 128)), row = query block, column = key block;
+ *                    any nonzero byte means "on".
+ *  mask_head_stride  elements between consecutive query heads' masks
+ *                    (head index b * H + h); 0 = one mask for every head.
+ * Rows left with no allowed key get O = 0, LSE = -inf and zero gradients.
+ * Errors as fa_fwd / fa_bwd, plus FA_ERR_INVALID_ARG for a null block_mask or a
+ * negative stride.  fa_bwd_workspace_size() applies unchanged.
+ */
+fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                             int Hkv, int N, int d, float scale, int causal, int window,
+                             const unsigned char* block_mask, long long mask_head_stride, fa_dtype dtype,
+                             void* stream);
+fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                             int H, int Hkv, int N, int d, float scale, int causal, int window,
+                             const unsigned char* block_mask, long long mask_head_stride, fa_dtype dtype,
+                             void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes (fp32 row terms
  * D_i = sum_k dO_ik O_ik, prescaled LSE, and for bf16 a float dQ accumulator).
  * Returns 0 for sizes fa_bwd would reject.

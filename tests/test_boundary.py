@@ -21,7 +21,7 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size"):
+              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse"):
         assert n in names
 
 
@@ -132,3 +132,15 @@ def test_splitkv_workspace_closed_form(L, B, H, N, d, S):
     assert L.fa_fwd_splitkv_workspace_size(B, H, N, d, S) == a256(S * B * H * nq2 * d * 4) + a256(S * B * H * nq2 * 16)
     assert L.fa_fwd_splitkv_workspace_size(B, H, N, d, 0) == 0
     assert L.fa_fwd_splitkv_workspace_size(B, H, N, d, 17) == 0
+
+
+def test_blocksparse_rejects_bad_arguments(L):
+    f = ctypes.c_float(0.125)
+    # null mask, negative stride, misaligned q, bad head ratio
+    assert L.fa_fwd_blocksparse(A, A, A, A, A, 1, 2, 1, 300, 64, f, 1, -1, None, 0, 0, None) == 1
+    assert L.fa_fwd_blocksparse(A, A, A, A, A, 1, 2, 1, 300, 64, f, 1, -1, A, -1, 0, None) == 1
+    assert L.fa_fwd_blocksparse(A + 8, A, A, A, A, 1, 2, 1, 300, 64, f, 1, -1, A, 0, 0, None) == 3
+    assert L.fa_fwd_blocksparse(A, A, A, A, A, 1, 3, 2, 300, 64, f, 1, -1, A, 0, 0, None) == 1
+    need = L.fa_bwd_workspace_size(1, 2, 300, 64, 0)
+    assert L.fa_bwd_blocksparse(*([A] * 10), need, 1, 2, 1, 300, 64, f, 1, -1, None, 0, 0, None) == 1
+    assert L.fa_bwd_blocksparse(*([A] * 10), need - 1, 1, 2, 1, 300, 64, f, 1, -1, A, 0, 0, None) == 4

@@ -44,3 +44,10 @@ def test_boosted_rows():
     norms = x["k"].reshape(-1, 128).norm(dim=1)
     big = int((norms > 40).sum())
     assert big == round(0.01 * 8 * 256)
+
+
+@pytest.mark.parametrize("N,causal,density", [(300, True, 0.5), (300, False, 0.5), (1000, True, 0.3), (129, False, 1.0)])
+def test_block_pairs_matches_brute_force(N, causal, density):
+    m = W.block_mask(N, density, 3, causal)
+    brute = int(ref.allowed(np.arange(N), np.arange(N), causal, -1, m).sum())
+    assert W.block_pairs(N, m, causal) == brute
