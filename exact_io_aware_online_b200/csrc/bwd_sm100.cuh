@@ -217,7 +217,7 @@ __device__ __forceinline__ void exp_cols64(const uint32_t (&sv)[64], const float
 }
 
 // ---------------------------------------------------------------- main kernel
-template <int D>
+template <int D, bool kMask>
 __global__ void __launch_bounds__(512, 1)
     bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -273,9 +273,10 @@ __global__ void __launch_bounds__(512, 1)
   // Work list: (query head hq of the group, query tile i) pairs in increasing
   // order, skipping blocks a block-sparse mask switches off.  Every role walks
   // it with its own QCursor, so all roles see the same sequence.
+  // (kMask: the block-sparse variant; the dense kernels compile no mask test.)
   const int bh0 = b * p.H + kh * p.g;
   auto active = [&](int hq, int i) {
-    return !p.bmask || p.bmask[(bh0 + hq) * p.bmask_hs + static_cast<long long>(i) * p.ntiles + j] != 0;
+    return !kMask || p.bmask[(bh0 + hq) * p.bmask_hs + static_cast<long long>(i) * p.ntiles + j] != 0;
   };
   struct QCursor {
     int hq, i;
@@ -286,16 +287,19 @@ __global__ void __launch_bounds__(512, 1)
         c.i = ilo;
         ++c.hq;
       }
-    } while (c.hq < p.g && !active(c.hq, c.i));
+    } while (kMask && c.hq < p.g && !active(c.hq, c.i));
     return c;
   };
   auto first = [&]() {
     QCursor c{0, ilo};
-    if (!active(0, ilo)) c = advance(c);
+    if (kMask && !active(0, ilo)) c = advance(c);
     return c;
   };
-  int total = 0;
-  for (QCursor c = first(); c.hq < p.g; c = advance(c)) ++total;
+  int total = (ihi - ilo + 1) * p.g;
+  if (kMask) {
+    total = 0;
+    for (QCursor c = first(); c.hq < p.g; c = advance(c)) ++total;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);

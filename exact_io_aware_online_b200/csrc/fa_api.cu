@@ -242,13 +242,18 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
       !make_tile_map(&tv, v, B * Hkv, N, D) || !make_tile_map(&tdo, dout, B * H, N, D) ||
       !make_tile_map(&tdk, dk, B * Hkv, N, D) || !make_tile_map(&tdv, dv, B * Hkv, N, D))
     return FA_ERR_CUDA;
-  if (!set_smem(fa::bwd_sm100_kernel<D>, C::kSmemBytes)) return FA_ERR_CUDA;
+  if (!set_smem(fa::bwd_sm100_kernel<D, false>, C::kSmemBytes) ||
+      !set_smem(fa::bwd_sm100_kernel<D, true>, C::kSmemBytes))
+    return FA_ERR_CUDA;
   const size_t rows = static_cast<size_t>(B) * H * p.Np;
   fa::bwd_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   const unsigned grid = static_cast<unsigned>(p.ntiles) * B * Hkv;
   mark_start(st);
-  fa::bwd_sm100_kernel<D><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
+  if (bmask)
+    fa::bwd_sm100_kernel<D, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
+  else
+    fa::bwd_sm100_kernel<D, false><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
   fa::bwd_dq_kernel<D><<<static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32)), 256, 0, st>>>(p);

@@ -331,6 +331,17 @@ __global__ void __launch_bounds__(384, 1)
       const bool block_off = kMask && !block_on(t, jcur);
       if (!(ok = mbar_wait(&s_full[t], jj & 1, abort_flag))) break;
       tc_fence_after();
+      if (kMask && block_off) {  // every weight of the tile is zero: store P = 0 and move on
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) z[i] = 0u;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_st16(tS + ch * 16, z);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+        continue;
+      }
       uint32_t sraw[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[c * 32]));
