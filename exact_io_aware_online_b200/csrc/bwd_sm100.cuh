@@ -557,6 +557,14 @@ __global__ void __launch_bounds__(512, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(dq_empty);  // TMEM tile free before the reductions are issued
+      if (C::kAliasDq && it + 1 < total) {
+        // Hold the row until the next dS has been written: the reductions then
+        // overlap the exponent phase instead of competing with the dS stores to
+        // shared memory.  Phase (it + 1) of ds_full cannot be overtaken: the
+        // phase after it needs dP^T of it + 2, which waits for this tile's
+        // dq_empty (the dQ tile aliases the dP^T columns when D = 128).
+        if (!(ok = mbar_wait(ds_full, (it + 1) & 1, abort_flag))) break;
+      }
 #pragma unroll
       for (int c = 0; c < D; c += 4) red_add_v4(dst + 32 * c, v[c], v[c + 1], v[c + 2], v[c + 3]);
     }
