@@ -41,6 +41,12 @@ What it computes, and where each step is stated:
   Reading: a 0/1 mask M over 128 x 128 blocks of the score matrix (per head or
   shared), and a key is allowed only if the causal / window predicate holds
   AND M[i // 128][j // 128] = 1.
+* Padding / variable lengths -- "FlashAttention" guide page, "Tiling through
+  SRAM": padding changes tiling details, not the rule.  Reading: batch entry b
+  holds L_b <= N valid tokens at the start of its [N, d] rows; keys >= L_b are
+  never attended to and padded query rows (>= L_b) give O = 0, LSE = -inf and
+  zero gradients, i.e. each batch entry is the attention of its first L_b
+  rows alone.
 * Fully masked rows (impossible in the shipped dense workloads, where the
   diagonal is always allowed; possible under a block mask) give O = 0,
   LSE = -inf and zero gradients.
@@ -135,20 +141,24 @@ def _head_mask(block_mask, b, h):
 
 
 def forward(q, k, v, scale: float, causal: bool = False, window: int = -1,
-            heads=None, row_block: int = 2048, block_mask=None):
+            heads=None, row_block: int = 2048, block_mask=None, seqlens=None):
     """O [B,H,N,d] and LSE [B,H,N] in fp64.
 
     q: [B,H,N,d]; k, v: [B,Hkv,N,d].  ``heads`` optionally restricts the work to
     a list of (b, h) pairs; other heads are left as NaN.  ``block_mask``: 0/1
     over 128 x 128 blocks, shape [nb, nb] (all heads) or [B, H, nb, nb].
+    ``seqlens``: optional [B] valid lengths (padding reading above).
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
-    b_, h_, _, n, d, g = _heads(q, k)
+    b_, h_, _, n_full, d, g = _heads(q, k)
     o = np.full(q.shape, np.nan)
     lse = np.full(q.shape[:3], np.nan)
     todo = heads if heads is not None else [(b, h) for b in range(b_) for h in range(h_)]
     for b, h in todo:
         kvh = h // g
+        n = n_full if seqlens is None else int(seqlens[b])
+        o[b, h, n:] = 0.0
+        lse[b, h, n:] = -np.inf
         for r0 in range(0, n, row_block):
             r1 = min(n, r0 + row_block)
             lo, hi = _key_range(r0, r1, n, causal, window)
@@ -167,7 +177,7 @@ def row_dot(p: np.ndarray, dp: np.ndarray) -> np.ndarray:
 
 
 def backward(q, k, v, do, scale: float, causal: bool = False, window: int = -1,
-             heads=None, row_block: int = 2048, block_mask=None):
+             heads=None, row_block: int = 2048, block_mask=None, seqlens=None):
     """dQ [B,H,N,d], dK and dV [B,Hkv,N,d] of L = sum(dO * O), in fp64.
 
     S and P are recomputed from Q and K (no saved forward state is used).
@@ -175,13 +185,15 @@ def backward(q, k, v, do, scale: float, causal: bool = False, window: int = -1,
     is NaN and dK/dV hold only the listed heads' contributions.
     """
     q, k, v, do = _as64(q), _as64(k), _as64(v), _as64(do)
-    b_, h_, _, n, d, g = _heads(q, k)
+    b_, h_, _, n_full, d, g = _heads(q, k)
     dq = np.full(q.shape, np.nan)
     dk = np.zeros(k.shape)
     dv = np.zeros(v.shape)
     todo = heads if heads is not None else [(b, h) for b in range(b_) for h in range(h_)]
     for b, h in todo:
         kvh = h // g
+        n = n_full if seqlens is None else int(seqlens[b])
+        dq[b, h, n:] = 0.0
         for r0 in range(0, n, row_block):
             r1 = min(n, r0 + row_block)
             lo, hi = _key_range(r0, r1, n, causal, window)

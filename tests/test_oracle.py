@@ -361,3 +361,37 @@ def test_block_mask_fully_masked_rows_and_per_head_masks():
     o_c, _ = ref.forward(q[:, :1], k[:, :1], v[:, :1], 0.5, causal=True, block_mask=bm[:, :1])
     o_cc, _ = ref.forward(q[:, :1], k[:, :1], v[:, :1], 0.5, causal=True)
     np.testing.assert_allclose(o_c, o_cc, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# Padding / variable lengths
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal,window", MODES)
+def test_seqlens_equal_truncated_problems(causal, window):
+    """Each batch entry with L_b valid tokens equals the attention of its
+    first L_b rows alone; padded rows are zero (LSE -inf), and whatever the
+    padding holds does not matter."""
+    b, h, n, d = 3, 2, 40, 5
+    q, k, v, do = (_rand((b, h, n, d), s) for s in (130, 131, 132, 133))
+    lens = [40, 17, 1]
+    o, lse = ref.forward(q, k, v, 0.6, causal, window, seqlens=lens)
+    gq, gk, gv = ref.backward(q, k, v, do, 0.6, causal, window, seqlens=lens)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for bi, L in enumerate(lens):  # garbage in the padding
+        q2[bi, :, L:] = 1e3
+        k2[bi, :, L:] = -1e3
+        v2[bi, :, L:] = 7.0
+    o2, lse2 = ref.forward(q2, k2, v2, 0.6, causal, window, seqlens=lens)
+    np.testing.assert_array_equal(o, o2)
+    np.testing.assert_array_equal(lse, lse2)
+    for bi, L in enumerate(lens):
+        ob, lb = ref.forward(q[bi:bi + 1, :, :L], k[bi:bi + 1, :, :L], v[bi:bi + 1, :, :L], 0.6, causal, window)
+        np.testing.assert_allclose(o[bi:bi + 1, :, :L], ob, atol=1e-14)
+        np.testing.assert_allclose(lse[bi:bi + 1, :, :L], lb, atol=1e-14)
+        assert np.all(o[bi, :, L:] == 0) and np.all(lse[bi, :, L:] == -np.inf)
+        g = ref.backward(q[bi:bi + 1, :, :L], k[bi:bi + 1, :, :L], v[bi:bi + 1, :, :L], do[bi:bi + 1, :, :L], 0.6,
+                         causal, window)
+        np.testing.assert_allclose(gq[bi:bi + 1, :, :L], g[0], atol=1e-13)
+        np.testing.assert_allclose(gk[bi:bi + 1, :, :L], g[1], atol=1e-13)
+        np.testing.assert_allclose(gv[bi:bi + 1, :, :L], g[2], atol=1e-13)
+        assert np.all(gq[bi, :, L:] == 0) and np.all(gk[bi, :, L:] == 0) and np.all(gv[bi, :, L:] == 0)
