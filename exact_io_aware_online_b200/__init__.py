@@ -14,7 +14,7 @@ import os
 import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
-           "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "LIB_PATH", "HEADER_PATH"]
+           "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "fwd_varlen", "bwd_varlen", "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_blocksparse.restype = i
     L.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, ll, i, vp]
     L.fa_bwd_blocksparse.restype = i
+    L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, vp]
+    L.fa_fwd_varlen.restype = i
+    L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
+    L.fa_bwd_varlen.restype = i
     _lib = L
     return L
 
@@ -222,6 +226,48 @@ def bwd_blocksparse(q, k, v, o, lse, do, block_mask, scale: float | None = None,
                                     ws.numel(), B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), mp, hs,
                                     code_t, _stream_ptr(q.device))
     _check(code, "fa_bwd_blocksparse")
+    return dq, dk, dv
+
+
+def _seqlens_ptr(seqlens, B):
+    import torch
+    if seqlens.dtype != torch.int32 or seqlens.numel() != B or not seqlens.is_cuda:
+        raise TypeError("seqlens must be a CUDA int32 tensor of B values")
+    return seqlens.contiguous().data_ptr()
+
+
+def fwd_varlen(q, k, v, seqlens, scale: float | None = None, causal: bool = False, window: int = -1,
+               out=None, lse=None):
+    """fwd() where batch entry b holds seqlens[b] valid tokens (padded layout)."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    code = lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                               B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window),
+                               _seqlens_ptr(seqlens, B), _dtype_code(q), _stream_ptr(q.device))
+    _check(code, "fa_fwd_varlen")
+    return o, l
+
+
+def bwd_varlen(q, k, v, o, lse, do, seqlens, scale: float | None = None, causal: bool = False, window: int = -1,
+               workspace=None, grads=None):
+    """bwd() of fwd_varlen()."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    code_t = _dtype_code(q)
+    need = bwd_workspace_size(B, H, N, d, code_t)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    code = lib().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
+                               B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window),
+                               _seqlens_ptr(seqlens, B), code_t, _stream_ptr(q.device))
+    _check(code, "fa_bwd_varlen")
     return dq, dk, dv
 
 

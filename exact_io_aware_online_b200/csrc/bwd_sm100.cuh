@@ -31,9 +31,10 @@
 // The two MMA streams touch disjoint TMEM regions (A: S^T and dV; B: dP^T, dK
 // and dQ), so each keeps its own order and a thread blocked pushing one
 // stream's instructions into a full tensor-core queue never delays the other.
-// Registers: 128 per thread at launch; the fourth warpgroup gives up 56 and
-// the drain takes them (128 + 128 + 184 + 72 = 4 * 128), so a drain thread
-// holds a whole dQ row and releases the TMEM tile before its reductions.
+// Registers: 128 per thread at launch; the fourth warpgroup drops to 64, the
+// compute warpgroups rise to 144 and the drain to 160 (144 + 144 + 160 + 64 =
+// 4 * 128), so a drain thread holds a whole dQ row and releases the TMEM tile
+// before its reductions.
 // The dQ accumulator uses a lane-interleaved layout (see dqacc_index) so that
 // the drain's vector reductions are coalesced: one warp instruction adds 512
 // contiguous bytes instead of touching 32 rows.
@@ -71,7 +72,12 @@ struct BwdParams {
   // [key block] per query head, bmask_hs elements apart (0: shared by all heads)
   const uint8_t* bmask;
   long long bmask_hs;
+  const int* seqlens;  // padded variable lengths (null: every batch entry has N rows)
 };
+
+__device__ __forceinline__ int valid_rows(const BwdParams& p, int b) {
+  return p.seqlens ? max(0, min(p.seqlens[b], p.N)) : p.N;
+}
 
 template <int D>
 struct BwdCfg {
@@ -102,7 +108,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   const int n = static_cast<int>(row % p.Np);
   float4* acc = reinterpret_cast<float4*>(p.dqacc + row * D);
   for (int x = lane; x < D / 4; x += 32) acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (n >= p.N) {
+  if (n >= valid_rows(p, static_cast<int>(bh / p.H))) {  // tile padding or a padded token
     if (lane == 0) {
       p.Drow[row] = 0.f;
       p.lse2[row] = INFINITY;
@@ -165,9 +171,10 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
     const int rr = f / (D / 4), u = f % (D / 4);
     const int n = 32 * g + rr;
     if (n >= p.N) continue;
+    const float sc = n < valid_rows(p, static_cast<int>(bh / p.H)) ? p.scale : 0.f;
     uint2 out;
-    out.x = pack_bf16x2(tile[rr][4 * u + 0] * p.scale, tile[rr][4 * u + 1] * p.scale);
-    out.y = pack_bf16x2(tile[rr][4 * u + 2] * p.scale, tile[rr][4 * u + 3] * p.scale);
+    out.x = pack_bf16x2(tile[rr][4 * u + 0] * sc, tile[rr][4 * u + 1] * sc);
+    out.y = pack_bf16x2(tile[rr][4 * u + 2] * sc, tile[rr][4 * u + 3] * sc);
     *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (bh * p.N + n) * D + 4 * u) = out;
   }
 }
@@ -264,7 +271,8 @@ __global__ void __launch_bounds__(512, 1)
   const int bkv = g0 + rem % gsz;
   const int b = bkv / p.Hkv, kh = bkv % p.Hkv;
   const int k0 = j * 128;
-  int ilo = 0, ihi = p.ntiles - 1;
+  const int Lb = valid_rows(p, b);
+  int ilo = 0, ihi = (max(Lb, 1) - 1) / 128;  // query tiles holding valid rows
   if (p.causal) ilo = j;
   if (p.window >= 0) {
     ilo = max(ilo, max(0, k0 - p.window) / 128);
@@ -295,8 +303,9 @@ __global__ void __launch_bounds__(512, 1)
     if (kMask && !active(0, ilo)) c = advance(c);
     return c;
   };
-  int total = (ihi - ilo + 1) * p.g;
-  if (kMask) {
+  const bool no_work = ilo > ihi || k0 >= Lb;  // nothing reaches this key tile
+  int total = no_work ? 0 : (ihi - ilo + 1) * p.g;
+  if (kMask && !no_work) {
     total = 0;
     for (QCursor c = first(); c.hq < p.g; c = advance(c)) ++total;
   }
@@ -328,7 +337,7 @@ __global__ void __launch_bounds__(512, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 12) {
-    regs_dec<72>();
+    regs_dec<64>();
     if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- producer
       prefetch_tmap(&tmQ);
@@ -452,6 +461,7 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ P and dS
+    regs_inc<144>();
     // Warpgroup w handles query columns [64w, 64w + 64); one key row per thread.
     const int w = warp >> 2, wl = warp & 3;
     const int r = wl * 32 + lane;
@@ -461,6 +471,8 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * w;
     const float sl2 = p.scale_log2;
     const int ds_chunk = w;  // 64-column (128-byte) block of the dS tile
+    const bool tile_valid = k0 + 127 < Lb;  // no padded key in this key tile
+    const bool key_valid = key < Lb;
     bool ok = true;
     QCursor cur = first();
     for (int it = 0; it < total; ++it, cur = advance(cur)) {
@@ -468,7 +480,7 @@ __global__ void __launch_bounds__(512, 1)
       const int q0 = cur.i * 128 + 64 * w;  // first query of my columns
       const float* Lv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes) + 64 * w;
       const float* Dv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes + 512) + 64 * w;
-      bool full = true;  // every (query, key) pair of my 64 columns allowed?
+      bool full = tile_valid;  // every (query, key) pair of my 64 columns allowed?
       if (p.causal) full = full && (k0 + 127 <= q0);
       if (p.window >= 0) full = full && (q0 + 63 - k0 <= p.window) && (k0 + 127 - q0 <= p.window);
       if (!(ok = mbar_wait(&q_full[s], (it / C::kStages) & 1, abort_flag))) break;  // LSE / D landed
@@ -487,7 +499,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
           const int q = q0 + c;
-          bool keep = true;
+          bool keep = key_valid;
           if (p.causal) keep = keep && key <= q;
           if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
           pv[c] = keep ? pv[c] : 0.f;
@@ -539,7 +551,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ drain, then dK/dV epilogue
-    regs_inc<184>();
+    regs_inc<160>();
     const int wl = warp & 3;
     const int r = wl * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;

@@ -109,7 +109,7 @@ inline size_t splitkv_ws_bytes(int B, int H, int N, int d, int splits) {
 template <int D>
 fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                    float scale, int causal, int window, cudaStream_t st, int splits = 0, void* ws = nullptr,
-                   const uint8_t* bmask = nullptr, long long bmask_hs = 0) {
+                   const uint8_t* bmask = nullptr, long long bmask_hs = 0, const int* seqlens = nullptr) {
   using C = fa::FwdCfg<D>;
   CUtensorMap tq, tk, tv, to;
   if (!make_tile_map(&tq, q, B * H, N, D) || !make_tile_map(&tk, k, B * Hkv, N, D) ||
@@ -134,6 +134,7 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   p.bmask = bmask;
   p.bmask_hs = bmask_hs;
   p.nbt = p.ntiles_kv;
+  p.seqlens = seqlens;
   {  // heads per group: Q, O and the (shared) K, V of a group within ~64 MiB of L2
     const double unit = static_cast<double>(N) * D * (4.0 + 4.0 / p.g);
     p.group = std::min(B * H, static_cast<int>(std::max(1.0, std::floor((64.0 * 1024 * 1024) / unit))));
@@ -167,11 +168,12 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
 template <int D>
 fa_status fwd_f32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                   float scale, int causal, int window, cudaStream_t st, const uint8_t* bmask = nullptr,
-                  long long bmask_hs = 0) {
+                  long long bmask_hs = 0, const int* seqlens = nullptr) {
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
   s.bmask = bmask;
   s.bmask_hs = bmask_hs;
   s.nbt = (N + 127) / 128;
+  s.seqlens = seqlens;
   s.q = static_cast<const float*>(q);
   s.k = static_cast<const float*>(k);
   s.v = static_cast<const float*>(v);
@@ -205,7 +207,8 @@ WsLayout ws_layout(int B, int H, int N, int d, fa_dtype dtype) {
 template <int D>
 fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                    void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
-                   int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0) {
+                   int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0,
+                   const int* seqlens = nullptr) {
   using C = fa::BwdCfg<D>;
   const WsLayout w = ws_layout(B, H, N, D, FA_BF16);
   uint8_t* wb = static_cast<uint8_t*>(ws);
@@ -230,6 +233,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   p.ntiles = p.Np / 128;
   p.bmask = bmask;
   p.bmask_hs = bmask_hs;
+  p.seqlens = seqlens;
   // kv heads per rasterisation group: keep each group's Q, dO, K, V and dQ
   // accumulator (about N*d*(4 + 8g) bytes per kv head) within ~64 MiB of L2.
   {
@@ -263,11 +267,13 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
 template <int D>
 fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                   void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
-                  int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0) {
+                  int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0,
+                  const int* seqlens = nullptr) {
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
   s.bmask = bmask;
   s.bmask_hs = bmask_hs;
   s.nbt = (N + 127) / 128;
+  s.seqlens = seqlens;
   s.q = static_cast<const float*>(q);
   s.k = static_cast<const float*>(k);
   s.v = static_cast<const float*>(v);
@@ -395,6 +401,47 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
                                block_mask, hs)
                  : bwd_f32<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
                                 block_mask, hs);
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                        int N, int d, float scale, int causal, int window, const int* seqlens, fa_dtype dtype,
+                        void* stream) {
+  if (!q || !k || !v || !o || !lse || !seqlens) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16)
+    return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, nullptr, 0,
+                                  seqlens)
+                   : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, nullptr, 0,
+                                   seqlens);
+  return d == 64 ? fwd_f32<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, nullptr, 0, seqlens)
+                 : fwd_f32<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, nullptr, 0, seqlens);
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H,
+                        int Hkv, int N, int d, float scale, int causal, int window, const int* seqlens,
+                        fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !seqlens) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < ws_layout(B, H, N, d, dtype).total) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16)
+    return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
+                                  nullptr, 0, seqlens)
+                   : bwd_bf16<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window,
+                                   st, nullptr, 0, seqlens);
+  return d == 64 ? bwd_f32<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
+                               nullptr, 0, seqlens)
+                 : bwd_f32<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
+                                nullptr, 0, seqlens);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype) {

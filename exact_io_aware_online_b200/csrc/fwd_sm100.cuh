@@ -53,6 +53,9 @@ struct FwdParams {
   int nbt;
   float* part_o;   // [splits][B*H][nq2][D] fp32 unnormalised O~, lane-interleaved (fwd_part_index)
   float4* part_m;  // [splits][B*H][nq2] {m (log2 units), l, l_bf16, 0}
+  // padded variable lengths (non-null): batch entry b has seqlens[b] valid rows;
+  // later keys are masked and later query rows give O = 0, LSE = -inf.
+  const int* seqlens;
 };
 
 // Partial-output layout: row n = 32 g + lane; the 16-byte unit u (columns
@@ -159,8 +162,10 @@ __global__ void __launch_bounds__(384, 1)
   const int b = bh / p.H, h = bh % p.H;
   const int kvh = b * p.Hkv + h / p.g;
   const int q0 = pair * 256;
-  const int qlast = min(q0 + 255, p.N - 1);
+  const int Lb = p.seqlens ? max(0, min(p.seqlens[b], p.N)) : p.N;  // valid rows of this batch entry
+  const int qlast = min(q0 + 255, Lb - 1);
   int jlo = 0, jhi = p.ntiles_kv - 1;
+  jhi = min(jhi, (max(Lb, 1) - 1) / 128);  // key tiles holding valid rows
   if (p.causal) jhi = min(jhi, qlast / 128);
   if (p.window >= 0) {
     jlo = max(0, q0 - p.window) / 128;
@@ -184,8 +189,9 @@ __global__ void __launch_bounds__(384, 1)
       while (j <= jhi && !block_on(0, j) && !block_on(1, j)) ++j;
     return j;
   };
-  int nkv = jhi - jlo + 1;
-  if (kMask) {
+  int nkv = max(0, jhi - jlo + 1);
+  if (qlast < q0) nkv = 0;  // the whole pair is padding
+  if (kMask && nkv > 0) {
     nkv = 0;
     for (int j = next_kv(jlo); j <= jhi; j = next_kv(j + 1)) ++nkv;
   }
@@ -349,14 +355,14 @@ __global__ void __launch_bounds__(384, 1)
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sraw[c]);
-      bool full = kv0 + 127 < p.N && !block_off;
+      bool full = kv0 + 127 < Lb && !block_off;
       if (p.causal) full = full && (kv0 + 127 <= tq0);
       if (p.window >= 0) full = full && (tq0 + 127 - kv0 <= p.window) && (kv0 + 127 - tq0 <= p.window);
       if (!full) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const int key = kv0 + c;
-          bool keep = key < p.N && !block_off;
+          bool keep = key < Lb && !block_off;
           if (p.causal) keep = keep && key <= qrow;
           if (p.window >= 0) keep = keep && abs(qrow - key) <= p.window;
           if (!keep) s[c] = -INFINITY;
@@ -422,13 +428,15 @@ __global__ void __launch_bounds__(384, 1)
           for (int u = 0; u < 8; ++u)
             *reinterpret_cast<uint4*>(dst + 32 * (c + 4 * u)) = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
         }
-        p.part_m[sbh * p.nq2 + n] = make_float4(m_used, l, lb, 0.f);
+        p.part_m[sbh * p.nq2 + n] = n < Lb ? make_float4(m_used, l, lb, 0.f) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
       }
     } else {
     if (ok && nkv > 0) ok = mbar_wait(&o_full[t], 0, abort_flag);
     if (ok) {
       tc_fence_after();
-      const float inv = (lb > 0.f) ? 1.f / lb : 0.f;
+      const bool pad_row = qrow >= Lb;
+      if (pad_row) l = 0.f;
+      const float inv = (lb > 0.f && !pad_row) ? 1.f / lb : 0.f;
       uint8_t* sO = sQ + t * C::kTileBytes;  // Q_t is no longer read
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {

@@ -38,7 +38,12 @@ struct SimtParams {
   const uint8_t* bmask;  // optional 0/1 mask per 128 x 128 block, [head][nbt][nbt]
   long long bmask_hs;    // elements between heads' masks (0: shared)
   int nbt;               // ceil(N / 128)
+  const int* seqlens;    // optional valid rows per batch entry (padded layout)
 };
+
+__device__ __forceinline__ int simt_valid_rows(const SimtParams& p, int b) {
+  return p.seqlens ? max(0, min(p.seqlens[b], p.N)) : p.N;
+}
 
 __device__ __forceinline__ bool keep_ij(int i, int j, int causal, int window) {
   return (!causal || j <= i) && (window < 0 || abs(i - j) <= window);
@@ -88,9 +93,10 @@ __global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
   const int kvh = b * p.Hkv + h / p.g;
-  const int r0 = blockIdx.x * kSimtRows, r1 = min(p.N, r0 + kSimtRows);
+  const int Lb = simt_valid_rows(p, b);
+  const int r0 = blockIdx.x * kSimtRows, r1 = min(Lb, r0 + kSimtRows);
   const int i = r0 + warp;
-  const bool active = i < p.N;
+  const bool active = i < Lb;
   const float* qrow = p.q + (static_cast<size_t>(bh) * p.N + (active ? i : 0)) * D;
   const float* kbase = p.k + static_cast<size_t>(kvh) * p.N * D;
   const float* vbase = p.v + static_cast<size_t>(kvh) * p.N * D;
@@ -102,7 +108,7 @@ __global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
   }
   float m = -INFINITY, l = 0.f;
   int lo, hi;
-  simt_key_range(r0, r1, p.N, p.causal, p.window, lo, hi);
+  simt_key_range(r0, max(r0, r1), Lb, p.causal, p.window, lo, hi);
   for (int kt = lo; kt < hi; kt += kSimtTile) {
     const int cnt = min(kSimtTile, hi - kt);
     __syncthreads();
@@ -132,7 +138,7 @@ __global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
       for (int e = 0; e < E; ++e) acc[e] = fmaf(pe, sV[jj][lane + 32 * e], acc[e]);
     }
   }
-  if (!active) return;
+  if (i >= p.N) return;  // padded rows (i >= Lb) end with l = 0: O = 0, LSE = -inf
   const float inv = l > 0.f ? 1.f / l : 0.f;
   float* orow = p.o_out + (static_cast<size_t>(bh) * p.N + i) * D;
 #pragma unroll
@@ -151,7 +157,8 @@ __global__ void __launch_bounds__(256) bwd_rowdot_f32_kernel(const SimtParams p)
 #pragma unroll
   for (int e = 0; e < E; ++e) s = fmaf(p.dout[row * D + lane + 32 * e], p.o[row * D + lane + 32 * e], s);
   s = warp_sum(s);
-  if (lane == 0) p.Drow[row] = s;
+  const int b = static_cast<int>(row / (static_cast<size_t>(p.H) * p.N));
+  if (lane == 0) p.Drow[row] = static_cast<int>(row % p.N) < simt_valid_rows(p, b) ? s : 0.f;
 }
 
 // dK, dV: one warp per key row of a kv head, summing over its query heads.
@@ -163,9 +170,10 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
   __shared__ float sL[kSimtTile], sD[kSimtTile];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bkv = blockIdx.y, b = bkv / p.Hkv, kh = bkv % p.Hkv;
-  const int c0 = blockIdx.x * kSimtRows, c1 = min(p.N, c0 + kSimtRows);
+  const int Lb = simt_valid_rows(p, b);
+  const int c0 = blockIdx.x * kSimtRows, c1 = min(Lb, c0 + kSimtRows);
   const int j = c0 + warp;
-  const bool active = j < p.N;
+  const bool active = j < Lb;
   const float* krow = p.k + (static_cast<size_t>(bkv) * p.N + (active ? j : 0)) * D;
   const float* vrow = p.v + (static_cast<size_t>(bkv) * p.N + (active ? j : 0)) * D;
   float kk[E], vv[E], dk[E], dv[E];
@@ -177,7 +185,7 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
     dv[e] = 0.f;
   }
   int lo, hi;
-  simt_query_range(c0, c1, p.N, p.causal, p.window, lo, hi);
+  simt_query_range(c0, max(c0, c1), Lb, p.causal, p.window, lo, hi);
   for (int hq = 0; hq < p.g; ++hq) {
     const int bh = b * p.H + kh * p.g + hq;
     const float* qbase = p.q + static_cast<size_t>(bh) * p.N * D;
@@ -216,7 +224,7 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
       }
     }
   }
-  if (!active) return;
+  if (j >= p.N) return;  // padded keys (j >= Lb) keep dk = dv = 0
   float* dkrow = p.dk + (static_cast<size_t>(bkv) * p.N + j) * D;
   float* dvrow = p.dv + (static_cast<size_t>(bkv) * p.N + j) * D;
 #pragma unroll
@@ -235,10 +243,11 @@ __global__ void __launch_bounds__(256) bwd_dq_f32_kernel(const SimtParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
   const int kvh = b * p.Hkv + h / p.g;
-  const int r0 = blockIdx.x * kSimtRows, r1 = min(p.N, r0 + kSimtRows);
+  const int Lb = simt_valid_rows(p, b);
+  const int r0 = blockIdx.x * kSimtRows, r1 = min(Lb, r0 + kSimtRows);
   const int i = r0 + warp;
-  const bool active = i < p.N;
-  const size_t row = static_cast<size_t>(bh) * p.N + (active ? i : 0);
+  const bool active = i < Lb;
+  const size_t row = static_cast<size_t>(bh) * p.N + (i < p.N ? i : 0);
   float q[E], dO[E], dq[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -250,7 +259,7 @@ __global__ void __launch_bounds__(256) bwd_dq_f32_kernel(const SimtParams p) {
   const float* kbase = p.k + static_cast<size_t>(kvh) * p.N * D;
   const float* vbase = p.v + static_cast<size_t>(kvh) * p.N * D;
   int lo, hi;
-  simt_key_range(r0, r1, p.N, p.causal, p.window, lo, hi);
+  simt_key_range(r0, max(r0, r1), Lb, p.causal, p.window, lo, hi);
   for (int kt = lo; kt < hi; kt += kSimtTile) {
     const int cnt = min(kSimtTile, hi - kt);
     __syncthreads();
@@ -276,7 +285,7 @@ __global__ void __launch_bounds__(256) bwd_dq_f32_kernel(const SimtParams p) {
       for (int e = 0; e < E; ++e) dq[e] = fmaf(ds, sK[jj][lane + 32 * e], dq[e]);
     }
   }
-  if (!active) return;
+  if (i >= p.N) return;  // padded rows (i >= Lb) keep dq = 0
 #pragma unroll
   for (int e = 0; e < E; ++e) p.dq[row * D + lane + 32 * e] = dq[e] * p.scale;
 }

@@ -121,6 +121,25 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
                              void* stream);
 
 /*
+ * Padded variable lengths: as fa_fwd / fa_bwd on the same [B, H, N, d]
+ * (and [B, Hkv, N, d]) layouts, where batch entry b holds only seqlens[b] valid
+ * tokens at the start of its rows ("FlashAttention" guide page, "Tiling through
+ * SRAM": padding changes tiling details, not the rule).  Keys at positions >=
+ * seqlens[b] are never attended to; query rows >= seqlens[b] get O = 0,
+ * LSE = -inf and zero dQ; key rows >= seqlens[b] get zero dK, dV.  Whatever the
+ * padding rows hold has no effect.  seqlens: device pointer to B int32 values,
+ * each clamped to [0, N] on the device; FA_ERR_INVALID_ARG if null.  Other
+ * arguments and errors as fa_fwd / fa_bwd.
+ */
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                        int N, int d, float scale, int causal, int window, const int* seqlens, fa_dtype dtype,
+                        void* stream);
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int H,
+                        int Hkv, int N, int d, float scale, int causal, int window, const int* seqlens,
+                        fa_dtype dtype, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes (fp32 row terms
  * D_i = sum_k dO_ik O_ik, prescaled LSE, and for bf16 a float dQ accumulator).
  * Returns 0 for sizes fa_bwd would reject.

@@ -21,7 +21,7 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse"):
+              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen"):
         assert n in names
 
 
@@ -144,3 +144,13 @@ def test_blocksparse_rejects_bad_arguments(L):
     need = L.fa_bwd_workspace_size(1, 2, 300, 64, 0)
     assert L.fa_bwd_blocksparse(*([A] * 10), need, 1, 2, 1, 300, 64, f, 1, -1, None, 0, 0, None) == 1
     assert L.fa_bwd_blocksparse(*([A] * 10), need - 1, 1, 2, 1, 300, 64, f, 1, -1, A, 0, 0, None) == 4
+
+
+def test_varlen_rejects_bad_arguments(L):
+    f = ctypes.c_float(0.125)
+    assert L.fa_fwd_varlen(A, A, A, A, A, 2, 2, 1, 300, 64, f, 1, -1, None, 0, None) == 1
+    assert L.fa_fwd_varlen(A, A, A, A, A, 2, 2, 1, 300, 96, f, 1, -1, A, 0, None) == 2
+    assert L.fa_fwd_varlen(A, A + 4, A, A, A, 2, 2, 1, 300, 64, f, 1, -1, A, 0, None) == 3
+    need = L.fa_bwd_workspace_size(2, 2, 300, 64, 1)
+    assert L.fa_bwd_varlen(*([A] * 10), need, 2, 2, 1, 300, 64, f, 1, -1, None, 1, None) == 1
+    assert L.fa_bwd_varlen(*([A] * 10), need - 1, 2, 2, 1, 300, 64, f, 1, -1, A, 1, None) == 4
