@@ -14,7 +14,8 @@ import os
 import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
-           "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "fwd_varlen", "bwd_varlen", "LIB_PATH", "HEADER_PATH"]
+           "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "fwd_varlen", "bwd_varlen", "fwd_strided", "bwd_strided",
+           "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -77,6 +78,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_varlen.restype = i
     L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
     L.fa_bwd_varlen.restype = i
+    L.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, vp]
+    L.fa_fwd_strided.restype = i
+    L.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
+    L.fa_bwd_strided.restype = i
     _lib = L
     return L
 
@@ -268,6 +273,62 @@ def bwd_varlen(q, k, v, o, lse, do, seqlens, scale: float | None = None, causal:
                                B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window),
                                _seqlens_ptr(seqlens, B), code_t, _stream_ptr(q.device))
     _check(code, "fa_bwd_varlen")
+    return dq, dk, dv
+
+
+class _Strides(ctypes.Structure):
+    """fa_strides of include/fa.h: element strides of the batch, head and row axes."""
+    _fields_ = [("batch", ctypes.c_longlong), ("head", ctypes.c_longlong), ("row", ctypes.c_longlong)]
+
+
+def _strides_of(*tensors):
+    arr = (_Strides * len(tensors))()
+    for n, t in enumerate(tensors):
+        if t.dim() != 4 or t.stride(3) != 1:
+            raise ValueError("tensors must be 4-D [B, heads, N, d] views with a contiguous last axis")
+        arr[n] = _Strides(t.stride(0), t.stride(1), t.stride(2))
+    return arr
+
+
+def fwd_strided(q, k, v, scale: float | None = None, causal: bool = False, window: int = -1, seqlens=None,
+                out=None, lse=None):
+    """fwd() on [B,H,N,d] / [B,Hkv,N,d] views of any layout with d contiguous
+    (e.g. x.transpose(1, 2) of a [B,N,H,d] buffer).  O takes q's layout unless
+    `out` is given; `seqlens` (optional) as in fwd_varlen()."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    st = _strides_of(q, k, v, o)
+    sp = _seqlens_ptr(seqlens, B) if seqlens is not None else None
+    code = lib().fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                ctypes.addressof(st), B, H, Hkv, N, d, float(scale), int(bool(causal)),
+                                int(window), sp, _dtype_code(q), _stream_ptr(q.device))
+    _check(code, "fa_fwd_strided")
+    return o, l
+
+
+def bwd_strided(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, window: int = -1,
+                seqlens=None, workspace=None, grads=None):
+    """bwd() of fwd_strided(); dq, dk, dv take the layouts of q, k, v unless
+    `grads` is given."""
+    import torch
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    code_t = _dtype_code(q)
+    need = bwd_workspace_size(B, H, N, d, code_t)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    st = _strides_of(q, k, v, o, do, dq, dk, dv)
+    sp = _seqlens_ptr(seqlens, B) if seqlens is not None else None
+    code = lib().fa_bwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ctypes.addressof(st),
+                                ws.data_ptr(), ws.numel(), B, H, Hkv, N, d, float(scale), int(bool(causal)),
+                                int(window), sp, code_t, _stream_ptr(q.device))
+    _check(code, "fa_bwd_strided")
     return dq, dk, dv
 
 

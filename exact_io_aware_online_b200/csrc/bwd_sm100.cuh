@@ -51,6 +51,8 @@
 // (c / 64) * 64 + (c % 64) / 2.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -75,6 +77,19 @@ struct BwdParams {
   const int* seqlens;  // padded variable lengths (null: every batch entry has N rows)
 };
 
+// Arguments of the strided-layout instantiations: element strides of O and dO
+// (read by the preprocess) and of dQ (written by the convert pass), and which
+// tensor maps are 4-D (column, row, head, batch entry) rather than 3-D (column,
+// row, batch entry * heads + head).  A separate type, so the contiguous
+// instantiations keep the plain BwdParams.
+struct BwdStridedParams : BwdParams {
+  Strides so, sdo, sdq;
+  unsigned map4;
+};
+constexpr unsigned kBMapQ = 1, kBMapK = 2, kBMapV = 4, kBMapDO = 8, kBMapDK = 16, kBMapDV = 32;
+template <bool kStrided>
+using BwdArgs = std::conditional_t<kStrided, BwdStridedParams, BwdParams>;
+
 __device__ __forceinline__ int valid_rows(const BwdParams& p, int b) {
   return p.seqlens ? max(0, min(p.seqlens[b], p.N)) : p.N;
 }
@@ -98,8 +113,8 @@ struct BwdCfg {
 };
 
 // ---------------------------------------------------------------- preprocess
-template <int D>
-__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
+template <int D, bool kStrided = false>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(blockIdx.x) * 8 + warp;  // over B*H*Np
   const size_t rows = static_cast<size_t>(p.B) * p.H * p.Np;
@@ -115,9 +130,17 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     }
     return;
   }
-  const size_t src = (bh * p.N + n) * D;
-  const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(p.o) + src / 2;
-  const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(p.dout) + src / 2;
+  const __nv_bfloat162* o2;
+  const __nv_bfloat162* d2;
+  if constexpr (kStrided) {
+    const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
+    o2 = reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.o) + p.so.row(b, h, n));
+    d2 = reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.dout) + p.sdo.row(b, h, n));
+  } else {
+    const size_t src = (bh * p.N + n) * D;
+    o2 = reinterpret_cast<const __nv_bfloat162*>(p.o) + src / 2;
+    d2 = reinterpret_cast<const __nv_bfloat162*>(p.dout) + src / 2;
+  }
   float s = 0.f;
   for (int x = lane; x < D / 2; x += 32) {
     const float2 a = __bfloat1622float2(o2[x]);
@@ -147,8 +170,8 @@ __device__ __forceinline__ size_t dqacc_unit(size_t bh, int Np, int g, int u) {
 // ---------------------------------------------------------------- dQ convert
 // One block per 32-row group: coalesced reads of the interleaved accumulator,
 // a transpose through shared memory, coalesced bf16 row writes of scale * acc.
-template <int D>
-__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
+template <int D, bool kStrided = false>
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs<kStrided> p) {
   __shared__ float tile[32][D + 4];
   const int groups = p.Np / 32;
   const size_t bh = blockIdx.x / groups;
@@ -175,7 +198,12 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdParams p) {
     uint2 out;
     out.x = pack_bf16x2(tile[rr][4 * u + 0] * sc, tile[rr][4 * u + 1] * sc);
     out.y = pack_bf16x2(tile[rr][4 * u + 2] * sc, tile[rr][4 * u + 3] * sc);
-    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (bh * p.N + n) * D + 4 * u) = out;
+    long long at;
+    if constexpr (kStrided)
+      at = p.sdq.row(static_cast<int>(bh / p.H), static_cast<int>(bh % p.H), n) + 4 * u;
+    else
+      at = static_cast<long long>((bh * p.N + n) * D + 4 * u);
+    *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + at) = out;
   }
 }
 
@@ -224,12 +252,12 @@ __device__ __forceinline__ void exp_cols64(const uint32_t (&sv)[64], const float
 }
 
 // ---------------------------------------------------------------- main kernel
-template <int D, bool kMask>
+template <int D, bool kMask, bool kStrided = false>
 __global__ void __launch_bounds__(512, 1)
     bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                      const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                     const BwdParams p) {
+                     const BwdArgs<kStrided> p) {
   using C = BwdCfg<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   if (smem_u32(smem_raw) & 1023u) {  // layout below assumes a 1024-aligned window
@@ -346,8 +374,13 @@ __global__ void __launch_bounds__(512, 1)
       prefetch_tmap(&tmdO);
       mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
       for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, k0, bkv);
-        tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, k0, bkv);
+        if constexpr (kStrided) {
+          tma_load_tile(&tmK, p.map4 & kBMapK, kv_full, sK + c * 16384, c * 64, k0, bkv, kh, b);
+          tma_load_tile(&tmV, p.map4 & kBMapV, kv_full, sV + c * 16384, c * 64, k0, bkv, kh, b);
+        } else {
+          tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, k0, bkv);
+          tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, k0, bkv);
+        }
       }
       int issued[C::kStages];
 #pragma unroll
@@ -360,8 +393,15 @@ __global__ void __launch_bounds__(512, 1)
         const int row0 = cur.i * 128, bh = bh0 + cur.hq;
         uint8_t* st = sStage + s * 2 * C::kTileBytes;
         for (int c = 0; c < C::kChunks; ++c) {
-          tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
-          tma_load_3d(&tmdO, &q_full[s], st + C::kTileBytes + c * 16384, c * 64, row0, bh);
+          if constexpr (kStrided) {
+            const int hq = kh * p.g + cur.hq;
+            tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, row0, bh, hq, b);
+            tma_load_tile(&tmdO, p.map4 & kBMapDO, &q_full[s], st + C::kTileBytes + c * 16384, c * 64, row0, bh, hq,
+                          b);
+          } else {
+            tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
+            tma_load_3d(&tmdO, &q_full[s], st + C::kTileBytes + c * 16384, c * 64, row0, bh);
+          }
         }
         const size_t vrow = static_cast<size_t>(bh) * p.Np + row0;
         bulk_load(sVec + s * C::kVecBytes, p.lse2 + vrow, 512, &q_full[s]);
@@ -606,8 +646,13 @@ __global__ void __launch_bounds__(512, 1)
     mbar_arrive(epi_bar);
     if (ok && r == 0 && mbar_wait(epi_bar, 0, abort_flag)) {
       for (int c = 0; c < C::kChunks; ++c) {
-        tma_store_3d(&tmdV, sV + c * 16384, c * 64, k0, bkv);
-        tma_store_3d(&tmdK, sK + c * 16384, c * 64, k0, bkv);
+        if constexpr (kStrided) {
+          tma_store_tile(&tmdV, p.map4 & kBMapDV, sV + c * 16384, c * 64, k0, bkv, kh, b);
+          tma_store_tile(&tmdK, p.map4 & kBMapDK, sK + c * 16384, c * 64, k0, bkv, kh, b);
+        } else {
+          tma_store_3d(&tmdV, sV + c * 16384, c * 64, k0, bkv);
+          tma_store_3d(&tmdK, sK + c * 16384, c * 64, k0, bkv);
+        }
       }
       bulk_commit();
       bulk_wait0();

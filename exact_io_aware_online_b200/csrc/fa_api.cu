@@ -64,18 +64,84 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// A [heads, N, d] bf16 tensor seen in 128-row x 64-column boxes with the
-// 128-byte swizzle (the layout the UMMA descriptors expect).
-bool make_tile_map(CUtensorMap* m, const void* ptr, int heads, int N, int d) {
+// A [B, heads, N, d] bf16 tensor (d contiguous, other axes at the given element
+// strides) in 128-row x 64-column boxes with the 128-byte swizzle (the layout
+// the UMMA descriptors expect).  When the batch axis steps exactly over all
+// heads (every contiguous layout, and slices of longer buffers) the two axes
+// merge and the map is 3-D (d, N, B * heads): the TMA unit serves those boxes
+// measurably faster than 4-D ones.  Otherwise (e.g. [B, N, H, d]) it is 4-D
+// (d, N, heads, B); *four reports which.  Rows past N are zero-filled on load
+// and clipped on store, so a tile never reaches another head's or batch
+// entry's rows whatever the strides.
+bool make_tile_map(CUtensorMap* m, const void* ptr, int B, int heads, int N, int d, const fa::Strides& s,
+                   bool* four) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(heads)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(N) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+  *four = !(B == 1 || s.b == static_cast<long long>(heads) * s.h);
+  const int rank = *four ? 4 : 3;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(*four ? heads : static_cast<long long>(B) * heads),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(s.n) * 2, static_cast<cuuint64_t>(s.h) * 2,
+                           static_cast<cuuint64_t>(s.b) * 2};
+  cuuint32_t box[4] = {64, 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Element strides of every tensor argument of one call.
+struct Layouts {
+  fa::Strides q, k, v, o, dout, dq, dk, dv;
+};
+
+Layouts contiguous_layouts(int B, int H, int Hkv, int N, int d) {
+  (void)B;
+  const fa::Strides qs = fa::contiguous_strides(H, N, d), ks = fa::contiguous_strides(Hkv, N, d);
+  return Layouts{qs, ks, ks, qs, qs, qs, ks, ks};
+}
+
+// True when the first n layouts (in q, k, v, o, dout, dq, dk, dv order) equal
+// those of b: such calls take the plain (contiguous) kernels.
+bool same_layouts(const Layouts& a, const Layouts& b, int n) {
+  const fa::Strides* x[8] = {&a.q, &a.k, &a.v, &a.o, &a.dout, &a.dq, &a.dk, &a.dv};
+  const fa::Strides* y[8] = {&b.q, &b.k, &b.v, &b.o, &b.dout, &b.dq, &b.dk, &b.dv};
+  for (int t = 0; t < n; ++t)
+    if (x[t]->b != y[t]->b || x[t]->h != y[t]->h || x[t]->n != y[t]->n) return false;
+  return true;
+}
+
+// Caller-supplied strides.  Every stride must be positive, a multiple of 16
+// bytes and below 2^40 bytes (the tensor-map limits); an axis of extent 1 has
+// its stride replaced by the row stride (it is never stepped).  Output layouts
+// must be one-to-one: sorted by stride, each axis must step past the whole
+// extent of the axes inside it, so that no two output elements share an address.
+fa_status check_strides(const fa::Strides& s, int B, int heads, int N, int d, int esize, bool output,
+                        fa::Strides* out) {
+  fa::Strides t = s;
+  if (t.n <= 0) return FA_ERR_INVALID_ARG;
+  if (B == 1) t.b = t.n;
+  if (heads == 1) t.h = t.n;
+  const long long lim = (1LL << 40) / esize;
+  for (long long x : {t.b, t.h, t.n}) {
+    if (x <= 0 || x >= lim) return FA_ERR_INVALID_ARG;
+    if ((x * esize) % 16 != 0) return FA_ERR_MISALIGNED;
+  }
+  if (output) {
+    struct Axis {
+      long long stride, extent;
+    } ax[3] = {{t.n, N}, {t.h, heads}, {t.b, B}};
+    std::sort(ax, ax + 3, [](const Axis& a, const Axis& b) { return a.stride < b.stride; });
+    long long span = d;  // elements covered by the axes already placed
+    for (const Axis& a : ax) {
+      if (a.extent == 1) continue;
+      if (a.stride < span) return FA_ERR_INVALID_ARG;
+      span = a.stride * a.extent;
+    }
+  }
+  *out = t;
+  return FA_OK;
 }
 
 template <typename K>
@@ -105,19 +171,25 @@ inline size_t splitkv_ws_bytes(int B, int H, int N, int d, int splits) {
 }
 
 // splits == 0: the plain forward; splits >= 1: split-KV partials into `ws`
-// followed by the merge kernel.
+// followed by the merge kernel.  L: non-null for a layout other than the
+// contiguous one (then no splits and no block mask); those calls run the
+// strided instantiation, the contiguous ones the plain kernels.
 template <int D>
 fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
-                   float scale, int causal, int window, cudaStream_t st, int splits = 0, void* ws = nullptr,
-                   const uint8_t* bmask = nullptr, long long bmask_hs = 0, const int* seqlens = nullptr) {
+                   float scale, int causal, int window, cudaStream_t st, const Layouts* L = nullptr, int splits = 0,
+                   void* ws = nullptr, const uint8_t* bmask = nullptr, long long bmask_hs = 0,
+                   const int* seqlens = nullptr) {
   using C = fa::FwdCfg<D>;
+  const Layouts lay = L ? *L : contiguous_layouts(B, H, Hkv, N, D);
   CUtensorMap tq, tk, tv, to;
-  if (!make_tile_map(&tq, q, B * H, N, D) || !make_tile_map(&tk, k, B * Hkv, N, D) ||
-      !make_tile_map(&tv, v, B * Hkv, N, D) || !make_tile_map(&to, o, B * H, N, D))
+  bool f4[4];
+  if (!make_tile_map(&tq, q, B, H, N, D, lay.q, &f4[0]) || !make_tile_map(&tk, k, B, Hkv, N, D, lay.k, &f4[1]) ||
+      !make_tile_map(&tv, v, B, Hkv, N, D, lay.v, &f4[2]) || !make_tile_map(&to, o, B, H, N, D, lay.o, &f4[3]))
     return FA_ERR_CUDA;
   if (!set_smem(fa::fwd_sm100_kernel<D, false, false>, C::kSmemBytes) ||
       !set_smem(fa::fwd_sm100_kernel<D, true, false>, C::kSmemBytes) ||
-      !set_smem(fa::fwd_sm100_kernel<D, false, true>, C::kSmemBytes))
+      !set_smem(fa::fwd_sm100_kernel<D, false, true>, C::kSmemBytes) ||
+      !set_smem(fa::fwd_sm100_kernel<D, false, false, true>, C::kSmemBytes))
     return FA_ERR_CUDA;
   fa::FwdParams p{};
   p.lse = lse;
@@ -142,6 +214,17 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
     p.group = std::min(p.group, B * H);
   }
   const unsigned grid = static_cast<unsigned>(p.npairs) * B * H;
+  if (L) {
+    if (splits != 0 || bmask) return FA_ERR_UNSUPPORTED;
+    fa::FwdStridedParams ps{};
+    static_cast<fa::FwdParams&>(ps) = p;
+    ps.map4 = (f4[0] ? fa::kMapQ : 0u) | (f4[1] ? fa::kMapK : 0u) | (f4[2] ? fa::kMapV : 0u) |
+              (f4[3] ? fa::kMapO : 0u);
+    mark_start(st);
+    fa::fwd_sm100_kernel<D, false, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, ps);
+    mark_stop(st);
+    return launched();
+  }
   if (splits == 0) {
     mark_start(st);
     if (bmask)
@@ -165,11 +248,23 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   return launched();
 }
 
+void set_simt_strides(fa::SimtParams& s, const Layouts& L) {
+  s.sq = L.q;
+  s.sk = L.k;
+  s.sv = L.v;
+  s.so = L.o;
+  s.sdo = L.dout;
+  s.sdq = L.dq;
+  s.sdk = L.dk;
+  s.sdv = L.dv;
+}
+
 template <int D>
 fa_status fwd_f32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
-                  float scale, int causal, int window, cudaStream_t st, const uint8_t* bmask = nullptr,
-                  long long bmask_hs = 0, const int* seqlens = nullptr) {
+                  float scale, int causal, int window, cudaStream_t st, const Layouts* L = nullptr,
+                  const uint8_t* bmask = nullptr, long long bmask_hs = 0, const int* seqlens = nullptr) {
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
+  set_simt_strides(s, L ? *L : contiguous_layouts(B, H, Hkv, N, D));
   s.bmask = bmask;
   s.bmask_hs = bmask_hs;
   s.nbt = (N + 127) / 128;
@@ -207,10 +302,11 @@ WsLayout ws_layout(int B, int H, int N, int d, fa_dtype dtype) {
 template <int D>
 fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                    void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
-                   int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0,
-                   const int* seqlens = nullptr) {
+                   int window, cudaStream_t st, const Layouts* L = nullptr, const uint8_t* bmask = nullptr,
+                   long long bmask_hs = 0, const int* seqlens = nullptr) {
   using C = fa::BwdCfg<D>;
   const WsLayout w = ws_layout(B, H, N, D, FA_BF16);
+  const Layouts lay = L ? *L : contiguous_layouts(B, H, Hkv, N, D);
   uint8_t* wb = static_cast<uint8_t*>(ws);
   fa::BwdParams p{};
   p.lse = lse;
@@ -242,17 +338,40 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
     p.group = std::min(p.group, B * Hkv);
   }
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
-  if (!make_tile_map(&tq, q, B * H, N, D) || !make_tile_map(&tk, k, B * Hkv, N, D) ||
-      !make_tile_map(&tv, v, B * Hkv, N, D) || !make_tile_map(&tdo, dout, B * H, N, D) ||
-      !make_tile_map(&tdk, dk, B * Hkv, N, D) || !make_tile_map(&tdv, dv, B * Hkv, N, D))
+  bool f4[6];
+  if (!make_tile_map(&tq, q, B, H, N, D, lay.q, &f4[0]) || !make_tile_map(&tk, k, B, Hkv, N, D, lay.k, &f4[1]) ||
+      !make_tile_map(&tv, v, B, Hkv, N, D, lay.v, &f4[2]) ||
+      !make_tile_map(&tdo, dout, B, H, N, D, lay.dout, &f4[3]) ||
+      !make_tile_map(&tdk, dk, B, Hkv, N, D, lay.dk, &f4[4]) || !make_tile_map(&tdv, dv, B, Hkv, N, D, lay.dv, &f4[5]))
     return FA_ERR_CUDA;
   if (!set_smem(fa::bwd_sm100_kernel<D, false>, C::kSmemBytes) ||
-      !set_smem(fa::bwd_sm100_kernel<D, true>, C::kSmemBytes))
+      !set_smem(fa::bwd_sm100_kernel<D, true>, C::kSmemBytes) ||
+      !set_smem(fa::bwd_sm100_kernel<D, false, true>, C::kSmemBytes))
     return FA_ERR_CUDA;
   const size_t rows = static_cast<size_t>(B) * H * p.Np;
-  fa::bwd_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(p);
-  if (launched() != FA_OK) return FA_ERR_CUDA;
+  const unsigned pre_grid = static_cast<unsigned>((rows + 7) / 8);
   const unsigned grid = static_cast<unsigned>(p.ntiles) * B * Hkv;
+  const unsigned dq_grid = static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32));
+  if (L) {
+    if (bmask) return FA_ERR_UNSUPPORTED;
+    fa::BwdStridedParams ps{};
+    static_cast<fa::BwdParams&>(ps) = p;
+    ps.so = lay.o;
+    ps.sdo = lay.dout;
+    ps.sdq = lay.dq;
+    ps.map4 = (f4[0] ? fa::kBMapQ : 0u) | (f4[1] ? fa::kBMapK : 0u) | (f4[2] ? fa::kBMapV : 0u) |
+              (f4[3] ? fa::kBMapDO : 0u) | (f4[4] ? fa::kBMapDK : 0u) | (f4[5] ? fa::kBMapDV : 0u);
+    fa::bwd_pre_kernel<D, true><<<pre_grid, 256, 0, st>>>(ps);
+    if (launched() != FA_OK) return FA_ERR_CUDA;
+    mark_start(st);
+    fa::bwd_sm100_kernel<D, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, ps);
+    mark_stop(st);
+    if (launched() != FA_OK) return FA_ERR_CUDA;
+    fa::bwd_dq_kernel<D, true><<<dq_grid, 256, 0, st>>>(ps);
+    return launched();
+  }
+  fa::bwd_pre_kernel<D><<<pre_grid, 256, 0, st>>>(p);
+  if (launched() != FA_OK) return FA_ERR_CUDA;
   mark_start(st);
   if (bmask)
     fa::bwd_sm100_kernel<D, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
@@ -260,16 +379,17 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
     fa::bwd_sm100_kernel<D, false><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
   mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
-  fa::bwd_dq_kernel<D><<<static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32)), 256, 0, st>>>(p);
+  fa::bwd_dq_kernel<D><<<dq_grid, 256, 0, st>>>(p);
   return launched();
 }
 
 template <int D>
 fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                   void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
-                  int window, cudaStream_t st, const uint8_t* bmask = nullptr, long long bmask_hs = 0,
-                  const int* seqlens = nullptr) {
+                  int window, cudaStream_t st, const Layouts* L = nullptr, const uint8_t* bmask = nullptr,
+                  long long bmask_hs = 0, const int* seqlens = nullptr) {
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
+  set_simt_strides(s, L ? *L : contiguous_layouts(B, H, Hkv, N, D));
   s.bmask = bmask;
   s.bmask_hs = bmask_hs;
   s.nbt = (N + 127) / 128;
@@ -296,6 +416,50 @@ fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, co
   dim3 gq((N + fa::kSimtRows - 1) / fa::kSimtRows, B * H);
   fa::bwd_dq_f32_kernel<D><<<gq, 32 * fa::kSimtRows, 0, st>>>(s);
   return launched();
+}
+
+// dtype / head-dimension dispatch shared by every entry point (arguments
+// already checked).
+fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
+                  int d, float scale, int causal, int window, fa_dtype dtype, void* stream, const Layouts* L,
+                  int splits = 0, void* ws = nullptr, const uint8_t* bmask = nullptr, long long hs = 0,
+                  const int* seqlens = nullptr) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16)
+    return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, L, splits, ws, bmask, hs,
+                                  seqlens)
+                   : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, L, splits, ws, bmask,
+                                   hs, seqlens);
+  if (splits != 0) return FA_ERR_UNSUPPORTED;
+  return d == 64 ? fwd_f32<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, L, bmask, hs, seqlens)
+                 : fwd_f32<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, L, bmask, hs, seqlens);
+}
+
+fa_status run_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, int d, float scale, int causal,
+                  int window, fa_dtype dtype, void* stream, const Layouts* L, const uint8_t* bmask = nullptr,
+                  long long hs = 0, const int* seqlens = nullptr) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == FA_BF16)
+    return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, ws, B, H, Hkv, N, scale, causal, window, st, L,
+                                  bmask, hs, seqlens)
+                   : bwd_bf16<128>(q, k, v, o, dout, lse, dq, dk, dv, ws, B, H, Hkv, N, scale, causal, window, st, L,
+                                   bmask, hs, seqlens);
+  return d == 64 ? bwd_f32<64>(q, k, v, o, dout, lse, dq, dk, dv, ws, B, H, Hkv, N, scale, causal, window, st, L,
+                               bmask, hs, seqlens)
+                 : bwd_f32<128>(q, k, v, o, dout, lse, dq, dk, dv, ws, B, H, Hkv, N, scale, causal, window, st, L,
+                                bmask, hs, seqlens);
+}
+
+fa_status check_bwd_buffers(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                            const float* lse, const void* dq, const void* dk, const void* dv, const void* workspace,
+                            size_t ws_bytes, int B, int H, int N, int d, fa_dtype dtype) {
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < ws_layout(B, H, N, d, dtype).total) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  return FA_OK;
 }
 
 }  // namespace
@@ -328,12 +492,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == FA_BF16)
-    return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st)
-                   : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st);
-  return d == 64 ? fwd_f32<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st)
-                 : fwd_f32<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st);
+  return run_fwd(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 nullptr);
 }
 
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits) {
@@ -353,9 +513,8 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
   if (!workspace || ws_bytes < splitkv_ws_bytes(B, H, N, d, num_splits)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, num_splits, workspace)
-                 : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, num_splits, workspace);
+  return run_fwd(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 nullptr, num_splits, workspace);
 }
 
 fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -366,14 +525,8 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
   if (s != FA_OK) return s;
   if (mask_head_stride < 0) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == FA_BF16)
-    return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, block_mask,
-                                  mask_head_stride)
-                   : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, block_mask,
-                                   mask_head_stride);
-  return d == 64 ? fwd_f32<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, block_mask, mask_head_stride)
-                 : fwd_f32<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, block_mask, mask_head_stride);
+  return run_fwd(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 nullptr, 0, nullptr, block_mask, mask_head_stride);
 }
 
 fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -385,22 +538,10 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
   fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
   if (s != FA_OK) return s;
   if (mask_head_stride < 0) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_MISALIGNED;
-  if (!workspace || ws_bytes < ws_layout(B, H, N, d, dtype).total) return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const long long hs = mask_head_stride;
-  if (dtype == FA_BF16)
-    return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
-                                  block_mask, hs)
-                   : bwd_bf16<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window,
-                                   st, block_mask, hs);
-  return d == 64 ? bwd_f32<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
-                               block_mask, hs)
-                 : bwd_f32<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
-                                block_mask, hs);
+  s = check_bwd_buffers(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, N, d, dtype);
+  if (s != FA_OK) return s;
+  return run_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 nullptr, block_mask, mask_head_stride);
 }
 
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
@@ -410,14 +551,8 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, fl
   fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == FA_BF16)
-    return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, nullptr, 0,
-                                  seqlens)
-                   : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, 0, nullptr, nullptr, 0,
-                                   seqlens);
-  return d == 64 ? fwd_f32<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, nullptr, 0, seqlens)
-                 : fwd_f32<128>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, nullptr, 0, seqlens);
+  return run_fwd(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 nullptr, 0, nullptr, nullptr, 0, seqlens);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -427,21 +562,57 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !seqlens) return FA_ERR_INVALID_ARG;
   fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
   if (s != FA_OK) return s;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_MISALIGNED;
-  if (!workspace || ws_bytes < ws_layout(B, H, N, d, dtype).total) return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == FA_BF16)
-    return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
-                                  nullptr, 0, seqlens)
-                   : bwd_bf16<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window,
-                                   st, nullptr, 0, seqlens);
-  return d == 64 ? bwd_f32<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
-                               nullptr, 0, seqlens)
-                 : bwd_f32<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st,
-                                nullptr, 0, seqlens);
+  s = check_bwd_buffers(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, N, d, dtype);
+  if (s != FA_OK) return s;
+  return run_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 nullptr, nullptr, 0, seqlens);
+}
+
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse, const fa_strides* strides,
+                         int B, int H, int Hkv, int N, int d, float scale, int causal, int window, const int* seqlens,
+                         fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse || !strides) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  Layouts L = contiguous_layouts(B, H, Hkv, N, d);
+  const int es = dtype == FA_BF16 ? 2 : 4;
+  fa::Strides* dst[4] = {&L.q, &L.k, &L.v, &L.o};
+  const int heads[4] = {H, Hkv, Hkv, H};
+  for (int t = 0; t < 4; ++t) {
+    const fa::Strides in{strides[t].batch, strides[t].head, strides[t].row};
+    s = check_strides(in, B, heads[t], N, d, es, t == 3, dst[t]);
+    if (s != FA_OK) return s;
+  }
+  const Layouts C0 = contiguous_layouts(B, H, Hkv, N, d);
+  const bool contig = same_layouts(L, C0, 4);
+  return run_fwd(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, window, dtype, stream, contig ? nullptr : &L, 0,
+                 nullptr, nullptr, 0,
+                 seqlens);
+}
+
+fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, const fa_strides* strides, void* workspace,
+                         size_t ws_bytes, int B, int H, int Hkv, int N, int d, float scale, int causal, int window,
+                         const int* seqlens, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !strides) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  s = check_bwd_buffers(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, N, d, dtype);
+  if (s != FA_OK) return s;
+  Layouts L = contiguous_layouts(B, H, Hkv, N, d);
+  const int es = dtype == FA_BF16 ? 2 : 4;
+  fa::Strides* dst[8] = {&L.q, &L.k, &L.v, &L.o, &L.dout, &L.dq, &L.dk, &L.dv};
+  const int heads[8] = {H, Hkv, Hkv, H, H, H, Hkv, Hkv};
+  for (int t = 0; t < 8; ++t) {
+    const fa::Strides in{strides[t].batch, strides[t].head, strides[t].row};
+    s = check_strides(in, B, heads[t], N, d, es, t >= 5, dst[t]);
+    if (s != FA_OK) return s;
+  }
+  const Layouts C0 = contiguous_layouts(B, H, Hkv, N, d);
+  const bool contig = same_layouts(L, C0, 8);
+  return run_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 contig ? nullptr : &L, nullptr, 0, seqlens);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype) {
@@ -455,18 +626,10 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
   if (s != FA_OK) return s;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_MISALIGNED;
-  if (!workspace || ws_bytes < ws_layout(B, H, N, d, dtype).total) return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (dtype == FA_BF16)
-    return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st)
-                   : bwd_bf16<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window,
-                                   st);
-  return d == 64 ? bwd_f32<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st)
-                 : bwd_f32<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, scale, causal, window, st);
+  s = check_bwd_buffers(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, N, d, dtype);
+  if (s != FA_OK) return s;
+  return run_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
+                 nullptr);
 }
 
 fa_status fa_last_device_status(void* stream) {

@@ -29,6 +29,8 @@
 // units), which keeps every p <= 2^kTau and is exact after the final 1/l.
 #pragma once
 
+#include <type_traits>
+
 #include "sm100_ptx.cuh"
 
 namespace fa {
@@ -57,6 +59,17 @@ struct FwdParams {
   // later keys are masked and later query rows give O = 0, LSE = -inf.
   const int* seqlens;
 };
+
+// Arguments of the strided-layout instantiation: the same fields plus which
+// tensor maps are 4-D (column, row, head, batch entry) rather than 3-D (column,
+// row, batch entry * heads + head).  A separate type, so the contiguous
+// instantiations keep the plain FwdParams.
+struct FwdStridedParams : FwdParams {
+  unsigned map4;
+};
+constexpr unsigned kMapQ = 1, kMapK = 2, kMapV = 4, kMapO = 8;
+template <bool kStrided>
+using FwdArgs = std::conditional_t<kStrided, FwdStridedParams, FwdParams>;
 
 // Partial-output layout: row n = 32 g + lane; the 16-byte unit u (columns
 // 4u..4u+3) of 32 consecutive rows is contiguous, so a warp whose lane owns a
@@ -122,11 +135,11 @@ __device__ __forceinline__ void exp_row_to_tmem(const float (&s)[128], float sl2
   lb += b0 + b1;
 }
 
-template <int D, bool kSplit, bool kMask>
+template <int D, bool kSplit, bool kMask, bool kStrided = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                     const FwdParams p) {
+                     const FwdArgs<kStrided> p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -231,7 +244,11 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(&tmQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128, bh);
+            if constexpr (kStrided)
+              tma_load_tile(&tmQ, p.map4 & kMapQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128,
+                            bh, h, b);
+            else
+              tma_load_3d(&tmQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128, bh);
       }
       int issued[C::kStages];
 #pragma unroll
@@ -245,8 +262,13 @@ __global__ void __launch_bounds__(384, 1)
           if (!mbar_wait(&kv_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
           mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
           const CUtensorMap* m = which == 0 ? &tmK : &tmV;
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(m, &kv_full[s], sKV + s * C::kTileBytes + c * 16384, c * 64, kv0, kvh);
+          for (int c = 0; c < C::kChunks; ++c) {
+            if constexpr (kStrided)
+              tma_load_tile(m, p.map4 & (which == 0 ? kMapK : kMapV), &kv_full[s], sKV + s * C::kTileBytes + c * 16384,
+                            c * 64, kv0, kvh, h / p.g, b);
+            else
+              tma_load_3d(m, &kv_full[s], sKV + s * C::kTileBytes + c * 16384, c * 64, kv0, kvh);
+          }
           ++issued[s];
         }
       }
@@ -468,7 +490,12 @@ __global__ void __launch_bounds__(384, 1)
     // bounded wait below cannot be left short of arrivals by a live peer.
     mbar_arrive(&epi_bar[t]);
     if (ok && r == 0 && tq0 < p.N && mbar_wait(&epi_bar[t], 0, abort_flag)) {
-      for (int c = 0; c < C::kChunks; ++c) tma_store_3d(&tmO, sQ + t * C::kTileBytes + c * 16384, c * 64, tq0, bh);
+      for (int c = 0; c < C::kChunks; ++c) {
+        if constexpr (kStrided)
+          tma_store_tile(&tmO, p.map4 & kMapO, sQ + t * C::kTileBytes + c * 16384, c * 64, tq0, bh, h, b);
+        else
+          tma_store_3d(&tmO, sQ + t * C::kTileBytes + c * 16384, c * 64, tq0, bh);
+      }
       bulk_commit();
       bulk_wait_read0();
     }

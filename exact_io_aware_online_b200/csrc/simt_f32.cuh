@@ -17,6 +17,8 @@
 
 #include <stdint.h>
 
+#include "layout.cuh"
+
 namespace fa {
 
 struct SimtParams {
@@ -39,6 +41,9 @@ struct SimtParams {
   long long bmask_hs;    // elements between heads' masks (0: shared)
   int nbt;               // ceil(N / 128)
   const int* seqlens;    // optional valid rows per batch entry (padded layout)
+  // element strides (batch, head, row) of each [B, heads, N, D] tensor; o is
+  // also the layout of o_out
+  Strides sq, sk, sv, so, sdo, sdq, sdk, sdv;
 };
 
 __device__ __forceinline__ int simt_valid_rows(const SimtParams& p, int b) {
@@ -92,14 +97,14 @@ __global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
   __shared__ float sV[kSimtTile][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
-  const int kvh = b * p.Hkv + h / p.g;
+  const int kh = h / p.g;
   const int Lb = simt_valid_rows(p, b);
   const int r0 = blockIdx.x * kSimtRows, r1 = min(Lb, r0 + kSimtRows);
   const int i = r0 + warp;
   const bool active = i < Lb;
-  const float* qrow = p.q + (static_cast<size_t>(bh) * p.N + (active ? i : 0)) * D;
-  const float* kbase = p.k + static_cast<size_t>(kvh) * p.N * D;
-  const float* vbase = p.v + static_cast<size_t>(kvh) * p.N * D;
+  const float* qrow = p.q + p.sq.row(b, h, active ? i : 0);
+  const float* kbase = p.k + p.sk.row(b, kh, 0);
+  const float* vbase = p.v + p.sv.row(b, kh, 0);
   float q[E], acc[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -113,8 +118,8 @@ __global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
     const int cnt = min(kSimtTile, hi - kt);
     __syncthreads();
     for (int x = threadIdx.x; x < cnt * D; x += blockDim.x) {
-      sK[x / D][x % D] = kbase[static_cast<size_t>(kt) * D + x];
-      sV[x / D][x % D] = vbase[static_cast<size_t>(kt) * D + x];
+      sK[x / D][x % D] = kbase[static_cast<long long>(kt + x / D) * p.sk.n + x % D];
+      sV[x / D][x % D] = vbase[static_cast<long long>(kt + x / D) * p.sv.n + x % D];
     }
     __syncthreads();
     if (!active) continue;
@@ -140,7 +145,7 @@ __global__ void __launch_bounds__(256) fwd_simt_f32_kernel(const SimtParams p) {
   }
   if (i >= p.N) return;  // padded rows (i >= Lb) end with l = 0: O = 0, LSE = -inf
   const float inv = l > 0.f ? 1.f / l : 0.f;
-  float* orow = p.o_out + (static_cast<size_t>(bh) * p.N + i) * D;
+  float* orow = p.o_out + p.so.row(b, h, i);
 #pragma unroll
   for (int e = 0; e < E; ++e) orow[lane + 32 * e] = acc[e] * inv;
   if (lane == 0) p.lse_out[static_cast<size_t>(bh) * p.N + i] = l > 0.f ? m + logf(l) : -INFINITY;
@@ -153,12 +158,16 @@ __global__ void __launch_bounds__(256) bwd_rowdot_f32_kernel(const SimtParams p)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t row = static_cast<size_t>(blockIdx.x) * kSimtRows + warp;
   if (row >= static_cast<size_t>(p.B) * p.H * p.N) return;
+  const int n = static_cast<int>(row % p.N);
+  const int b = static_cast<int>(row / (static_cast<size_t>(p.H) * p.N));
+  const int h = static_cast<int>((row / p.N) % p.H);
+  const float* dorow = p.dout + p.sdo.row(b, h, n);
+  const float* orow = p.o + p.so.row(b, h, n);
   float s = 0.f;
 #pragma unroll
-  for (int e = 0; e < E; ++e) s = fmaf(p.dout[row * D + lane + 32 * e], p.o[row * D + lane + 32 * e], s);
+  for (int e = 0; e < E; ++e) s = fmaf(dorow[lane + 32 * e], orow[lane + 32 * e], s);
   s = warp_sum(s);
-  const int b = static_cast<int>(row / (static_cast<size_t>(p.H) * p.N));
-  if (lane == 0) p.Drow[row] = static_cast<int>(row % p.N) < simt_valid_rows(p, b) ? s : 0.f;
+  if (lane == 0) p.Drow[row] = n < simt_valid_rows(p, b) ? s : 0.f;
 }
 
 // dK, dV: one warp per key row of a kv head, summing over its query heads.
@@ -174,8 +183,8 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
   const int c0 = blockIdx.x * kSimtRows, c1 = min(Lb, c0 + kSimtRows);
   const int j = c0 + warp;
   const bool active = j < Lb;
-  const float* krow = p.k + (static_cast<size_t>(bkv) * p.N + (active ? j : 0)) * D;
-  const float* vrow = p.v + (static_cast<size_t>(bkv) * p.N + (active ? j : 0)) * D;
+  const float* krow = p.k + p.sk.row(b, kh, active ? j : 0);
+  const float* vrow = p.v + p.sv.row(b, kh, active ? j : 0);
   float kk[E], vv[E], dk[E], dv[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -188,14 +197,14 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
   simt_query_range(c0, max(c0, c1), Lb, p.causal, p.window, lo, hi);
   for (int hq = 0; hq < p.g; ++hq) {
     const int bh = b * p.H + kh * p.g + hq;
-    const float* qbase = p.q + static_cast<size_t>(bh) * p.N * D;
-    const float* obase = p.dout + static_cast<size_t>(bh) * p.N * D;
+    const float* qbase = p.q + p.sq.row(b, kh * p.g + hq, 0);
+    const float* obase = p.dout + p.sdo.row(b, kh * p.g + hq, 0);
     for (int it = lo; it < hi; it += kSimtTile) {
       const int cnt = min(kSimtTile, hi - it);
       __syncthreads();
       for (int x = threadIdx.x; x < cnt * D; x += blockDim.x) {
-        sQ[x / D][x % D] = qbase[static_cast<size_t>(it) * D + x];
-        sO[x / D][x % D] = obase[static_cast<size_t>(it) * D + x];
+        sQ[x / D][x % D] = qbase[static_cast<long long>(it + x / D) * p.sq.n + x % D];
+        sO[x / D][x % D] = obase[static_cast<long long>(it + x / D) * p.sdo.n + x % D];
       }
       for (int x = threadIdx.x; x < cnt; x += blockDim.x) {
         sL[x] = p.lse[static_cast<size_t>(bh) * p.N + it + x];
@@ -225,8 +234,8 @@ __global__ void __launch_bounds__(256) bwd_dkdv_f32_kernel(const SimtParams p) {
     }
   }
   if (j >= p.N) return;  // padded keys (j >= Lb) keep dk = dv = 0
-  float* dkrow = p.dk + (static_cast<size_t>(bkv) * p.N + j) * D;
-  float* dvrow = p.dv + (static_cast<size_t>(bkv) * p.N + j) * D;
+  float* dkrow = p.dk + p.sdk.row(b, kh, j);
+  float* dvrow = p.dv + p.sdv.row(b, kh, j);
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     dkrow[lane + 32 * e] = dk[e] * p.scale;
@@ -242,30 +251,31 @@ __global__ void __launch_bounds__(256) bwd_dq_f32_kernel(const SimtParams p) {
   __shared__ float sV[kSimtTile][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
-  const int kvh = b * p.Hkv + h / p.g;
+  const int kh = h / p.g;
   const int Lb = simt_valid_rows(p, b);
   const int r0 = blockIdx.x * kSimtRows, r1 = min(Lb, r0 + kSimtRows);
   const int i = r0 + warp;
   const bool active = i < Lb;
-  const size_t row = static_cast<size_t>(bh) * p.N + (i < p.N ? i : 0);
+  const int ir = i < p.N ? i : 0;
+  const size_t row = static_cast<size_t>(bh) * p.N + ir;  // LSE and D rows (contiguous)
   float q[E], dO[E], dq[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    q[e] = p.q[row * D + lane + 32 * e];
-    dO[e] = p.dout[row * D + lane + 32 * e];
+    q[e] = p.q[p.sq.row(b, h, ir) + lane + 32 * e];
+    dO[e] = p.dout[p.sdo.row(b, h, ir) + lane + 32 * e];
     dq[e] = 0.f;
   }
   const float L = p.lse[row], Dr = p.Drow[row];
-  const float* kbase = p.k + static_cast<size_t>(kvh) * p.N * D;
-  const float* vbase = p.v + static_cast<size_t>(kvh) * p.N * D;
+  const float* kbase = p.k + p.sk.row(b, kh, 0);
+  const float* vbase = p.v + p.sv.row(b, kh, 0);
   int lo, hi;
   simt_key_range(r0, max(r0, r1), Lb, p.causal, p.window, lo, hi);
   for (int kt = lo; kt < hi; kt += kSimtTile) {
     const int cnt = min(kSimtTile, hi - kt);
     __syncthreads();
     for (int x = threadIdx.x; x < cnt * D; x += blockDim.x) {
-      sK[x / D][x % D] = kbase[static_cast<size_t>(kt) * D + x];
-      sV[x / D][x % D] = vbase[static_cast<size_t>(kt) * D + x];
+      sK[x / D][x % D] = kbase[static_cast<long long>(kt + x / D) * p.sk.n + x % D];
+      sV[x / D][x % D] = vbase[static_cast<long long>(kt + x / D) * p.sv.n + x % D];
     }
     __syncthreads();
     if (!active) continue;
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(256) bwd_dq_f32_kernel(const SimtParams p) {
   }
   if (i >= p.N) return;  // padded rows (i >= Lb) keep dq = 0
 #pragma unroll
-  for (int e = 0; e < E; ++e) p.dq[row * D + lane + 32 * e] = dq[e] * p.scale;
+  for (int e = 0; e < E; ++e) p.dq[p.sdq.row(b, h, i) + lane + 32 * e] = dq[e] * p.scale;
 }
 
 }  // namespace fa

@@ -8,6 +8,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "layout.cuh"
+
 namespace fa {
 
 // Device status word: a bounded wait that gives up ORs a code in here.
@@ -83,6 +85,15 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap* map, uint64_t* ba
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
+// 4-D tiled TMA load: coordinates (column, row, head, batch entry).
+__device__ __forceinline__ void tma_load_4d(const CUtensorMap* map, uint64_t* bar, void* dst, int c0, int c1,
+                                            int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
 // 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -95,6 +106,30 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
                    reinterpret_cast<uint64_t>(map)),
                "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
                : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                             int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+// Tile of head idx = b * heads + h of a [B, heads, N, D] tensor: through a
+// 3-D map (column, row, idx) when the batch and head axes merge, else through a
+// 4-D map (column, row, h, b).
+__device__ __forceinline__ void tma_load_tile(const CUtensorMap* map, bool four, uint64_t* bar, void* dst, int c,
+                                              int row, int idx, int h, int b) {
+  if (four)
+    tma_load_4d(map, bar, dst, c, row, h, b);
+  else
+    tma_load_3d(map, bar, dst, c, row, idx);
+}
+__device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, bool four, const void* src, int c, int row,
+                                               int idx, int h, int b) {
+  if (four)
+    tma_store_4d(map, src, c, row, h, b);
+  else
+    tma_store_3d(map, src, c, row, idx);
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

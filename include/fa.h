@@ -140,6 +140,41 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
                         fa_dtype dtype, void* stream);
 
 /*
+ * Strided layouts: as fa_fwd_varlen / fa_bwd_varlen (seqlens may be NULL: every
+ * batch entry then has N valid rows), but each tensor argument may have any
+ * layout whose head dimension d is contiguous -- e.g. [B, N, H, d] ("BSHD",
+ * tokens outer, heads inner), a slice of a longer buffer, or rows with a
+ * padded pitch.  The same rule and outputs as fa_fwd / fa_bwd ("FlashAttention"
+ * guide page, "Tiling through SRAM": the layout only changes how tiles are
+ * addressed, and the tile schedule is the same).  lse stays [B, H, N]
+ * contiguous fp32.
+ *
+ * strides: host pointer to 4 (fwd: q, k, v, o) or 8 (bwd: q, k, v, o, dout, dq,
+ * dk, dv) fa_strides, in ELEMENTS: element (b, h, n, c) of a tensor is at
+ * b * batch + h * head + n * row + c.  The contiguous [B, H, N, d] layout is
+ * {H*N*d, N*d, d}; a [B, N, H, d] buffer seen as [B, H, N, d] is {N*H*d, d, H*d}.
+ * Rules (FA_ERR_INVALID_ARG unless noted): every stride > 0 and < 2^40 bytes;
+ * every stride times the element size a multiple of 16 bytes
+ * (FA_ERR_MISALIGNED); the stride of an axis of extent 1 (B == 1, or a single
+ * head) is ignored; an output layout (o, dq, dk, dv) must be one-to-one -- with
+ * its axes sorted by stride, each stride at least the span of the axes inside
+ * it (d for the innermost).  Inputs may overlap each other; outputs must not
+ * overlap inputs or each other (not checked).  Elements of an output buffer
+ * that no (b, h, n, c) maps to are never written.  Other arguments, errors and
+ * fa_bwd_workspace_size() as fa_fwd / fa_bwd.
+ */
+typedef struct {
+  long long batch, head, row; /* element strides; d is contiguous */
+} fa_strides;
+fa_status fa_fwd_strided(const void* q, const void* k, const void* v, void* o, float* lse,
+                         const fa_strides* strides, int B, int H, int Hkv, int N, int d, float scale, int causal,
+                         int window, const int* seqlens, fa_dtype dtype, void* stream);
+fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, const fa_strides* strides, void* workspace,
+                         size_t ws_bytes, int B, int H, int Hkv, int N, int d, float scale, int causal, int window,
+                         const int* seqlens, fa_dtype dtype, void* stream);
+
+/*
  * Bytes of device workspace fa_bwd needs for these sizes (fp32 row terms
  * D_i = sum_k dO_ik O_ik, prescaled LSE, and for bf16 a float dQ accumulator).
  * Returns 0 for sizes fa_bwd would reject.

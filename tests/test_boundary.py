@@ -21,7 +21,7 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen"):
+              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_strided", "fa_bwd_strided"):
         assert n in names
 
 
@@ -154,3 +154,58 @@ def test_varlen_rejects_bad_arguments(L):
     need = L.fa_bwd_workspace_size(2, 2, 300, 64, 1)
     assert L.fa_bwd_varlen(*([A] * 10), need, 2, 2, 1, 300, 64, f, 1, -1, None, 1, None) == 1
     assert L.fa_bwd_varlen(*([A] * 10), need - 1, 2, 2, 1, 300, 64, f, 1, -1, A, 1, None) == 4
+
+
+def _strides(rows):
+    arr = (fa._Strides * len(rows))()
+    for n, (b, h, r) in enumerate(rows):
+        arr[n] = fa._Strides(b, h, r)
+    return arr
+
+
+def test_strided_rejects_bad_arguments(L):
+    f = ctypes.c_float(0.125)
+    B, H, Hkv, N, d = 2, 4, 2, 300, 64
+    q = (H * N * d, N * d, d)          # contiguous [B, H, N, d]
+    kv = (Hkv * N * d, N * d, d)
+    bshd = (N * H * d, d, H * d)       # [B, N, H, d] seen as [B, H, N, d]
+
+    def fwd(rows, dtype=0, dd=d):
+        return L.fa_fwd_strided(A, A, A, A, A, ctypes.addressof(rows) if rows is not None else None,
+                                B, H, Hkv, N, dd, f, 1, -1, None, dtype, None)
+
+    assert fwd(None) == 1
+    assert fwd(_strides([q, kv, kv, (q[0], q[1], 0)])) == 1            # zero row stride
+    assert fwd(_strides([(q[0], q[1], -d), kv, kv, q])) == 1           # negative stride
+    assert fwd(_strides([q, kv, (kv[0], kv[1], d + 4), q])) == 3       # 8-byte pitch: not 16-byte aligned
+    assert fwd(_strides([q, kv, kv, (q[0], q[1], d // 2)])) == 1       # output rows overlap
+    assert fwd(_strides([q, kv, kv, (q[0], d, d)])) == 1               # output heads overlap rows
+    assert fwd(_strides([q, kv, kv, (N * d, N * d, d)])) == 1          # output batch entries overlap heads
+    assert fwd(_strides([q, kv, kv, (1 << 40, q[1], d)])) == 1         # beyond the tensor-map range
+    assert fwd(_strides([q, kv, kv, bshd]), dd=96) == 2                # d still 64 or 128
+    # fp32: strides must be multiples of 4 elements
+    assert fwd(_strides([q, kv, (kv[0], kv[1], d + 2), q]), dtype=1) == 3
+    need = L.fa_bwd_workspace_size(B, H, N, d, 0)
+    good = [q, kv, kv, q, q, q, kv, kv]
+
+    def bwd(rows, ws=need):
+        return L.fa_bwd_strided(*([A] * 9), ctypes.addressof(rows) if rows is not None else None, A, ws,
+                                B, H, Hkv, N, d, f, 1, -1, None, 0, None)
+
+    assert bwd(None) == 1
+    assert bwd(_strides(good), ws=need - 1) == 4
+    bad = list(good)
+    bad[6] = (kv[0], kv[1], d // 2)                                     # dk rows overlap
+    assert bwd(_strides(bad)) == 1
+    bad = list(good)
+    bad[4] = (q[0], q[1], d + 4)                                        # dout pitch misaligned
+    assert bwd(_strides(bad)) == 3
+
+
+def test_strided_helper_requires_contiguous_last_axis():
+    import torch
+    x = torch.zeros(1, 2, 8, 64).transpose(2, 3)
+    with pytest.raises(ValueError):
+        fa._strides_of(x)
+    st = fa._strides_of(torch.zeros(2, 8, 3, 64).transpose(1, 2))
+    assert (st[0].batch, st[0].head, st[0].row) == (8 * 3 * 64, 64, 3 * 64)
