@@ -50,6 +50,11 @@ What it computes, and where each step is stated:
 * Fully masked rows (impossible in the shipped dense workloads, where the
   diagonal is always allowed; possible under a block mask) give O = 0,
   LSE = -inf and zero gradients.
+* Fewer queries than keys (decode) -- "FlashAttention" guide page, "Key
+  takeaways": prefill and decode change the mapping, not the math.  Reading:
+  the Nq queries are the newest Nq tokens of a length-Nk sequence, so query i
+  sits at position Nk - Nq + i and the causal / window predicate is applied to
+  that position (forward only; Nq <= Nk).
 
 Implementation notes, none of which changes a value: rows are processed in
 blocks (each row's softmax is still computed over its whole key range at once),
@@ -142,27 +147,33 @@ def _head_mask(block_mask, b, h):
 
 def forward(q, k, v, scale: float, causal: bool = False, window: int = -1,
             heads=None, row_block: int = 2048, block_mask=None, seqlens=None):
-    """O [B,H,N,d] and LSE [B,H,N] in fp64.
+    """O [B,H,Nq,d] and LSE [B,H,Nq] in fp64.
 
-    q: [B,H,N,d]; k, v: [B,Hkv,N,d].  ``heads`` optionally restricts the work to
-    a list of (b, h) pairs; other heads are left as NaN.  ``block_mask``: 0/1
-    over 128 x 128 blocks, shape [nb, nb] (all heads) or [B, H, nb, nb].
-    ``seqlens``: optional [B] valid lengths (padding reading above).
+    q: [B,H,Nq,d]; k, v: [B,Hkv,Nk,d] with Nq <= Nk (Nq < Nk: decode reading
+    above).  ``heads`` optionally restricts the work to a list of (b, h) pairs;
+    other heads are left as NaN.  ``block_mask``: 0/1 over 128 x 128 blocks,
+    shape [nb, nb] (all heads) or [B, H, nb, nb].  ``seqlens``: optional [B]
+    valid lengths (padding reading above).  Both need Nq == Nk.
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
-    b_, h_, _, n_full, d, g = _heads(q, k)
+    b_, h_, _, nq_full, d, g = _heads(q, k)
+    nk_full = k.shape[2]
+    if nq_full > nk_full or (nq_full != nk_full and (seqlens is not None or block_mask is not None)):
+        raise ValueError("need Nq <= Nk, and Nq == Nk with seqlens or a block mask")
+    qoff = nk_full - nq_full  # position of query row 0
     o = np.full(q.shape, np.nan)
     lse = np.full(q.shape[:3], np.nan)
     todo = heads if heads is not None else [(b, h) for b in range(b_) for h in range(h_)]
     for b, h in todo:
         kvh = h // g
-        n = n_full if seqlens is None else int(seqlens[b])
-        o[b, h, n:] = 0.0
-        lse[b, h, n:] = -np.inf
-        for r0 in range(0, n, row_block):
-            r1 = min(n, r0 + row_block)
-            lo, hi = _key_range(r0, r1, n, causal, window)
-            rows, keys = np.arange(r0, r1), np.arange(lo, hi)
+        nq = nq_full if seqlens is None else int(seqlens[b])
+        nk = nk_full if seqlens is None else int(seqlens[b])
+        o[b, h, nq:] = 0.0
+        lse[b, h, nq:] = -np.inf
+        for r0 in range(0, nq, row_block):
+            r1 = min(nq, r0 + row_block)
+            lo, hi = _key_range(qoff + r0, qoff + r1, nk, causal, window)
+            rows, keys = np.arange(qoff + r0, qoff + r1), np.arange(lo, hi)
             p, m, l = attention_probs(q[b, h, r0:r1], k[b, kvh, lo:hi], scale,
                                       rows, keys, causal, window, _head_mask(block_mask, b, h))
             o[b, h, r0:r1] = p @ v[b, kvh, lo:hi]

@@ -395,3 +395,55 @@ def test_seqlens_equal_truncated_problems(causal, window):
         np.testing.assert_allclose(gk[bi:bi + 1, :, :L], g[1], atol=1e-13)
         np.testing.assert_allclose(gv[bi:bi + 1, :, :L], g[2], atol=1e-13)
         assert np.all(gq[bi, :, L:] == 0) and np.all(gk[bi, :, L:] == 0) and np.all(gv[bi, :, L:] == 0)
+
+
+# --------------------------------------------------------------------------
+# Fewer queries than keys (decode): query i sits at position Nk - Nq + i
+# ("FlashAttention" guide page, "Key takeaways": decode changes the mapping,
+# not the math).
+# --------------------------------------------------------------------------
+def test_decode_brute_force_tiny():
+    """Each query row written out with explicit loops: softmax over the keys its
+    position may see, then the weighted sum of V rows."""
+    nq, nk, d, scale = 2, 5, 3, 0.7
+    q, k, v = (_rand((1, 1, n, d), s) for n, s in ((nq, 140), (nk, 141), (nk, 142)))
+    for causal, window in ((True, -1), (False, 1), (True, 1), (False, -1)):
+        o, lse = ref.forward(q, k, v, scale, causal, window)
+        for i in range(nq):
+            pos = nk - nq + i
+            keys = [j for j in range(nk) if (not causal or j <= pos) and (window < 0 or abs(pos - j) <= window)]
+            s = [scale * sum(q[0, 0, i, c] * k[0, 0, j, c] for c in range(d)) for j in keys]
+            mx = max(s)
+            w = [math.exp(x - mx) for x in s]
+            tot = sum(w)
+            for c in range(d):
+                want = sum(wj * v[0, 0, j, c] for wj, j in zip(w, keys)) / tot
+                assert abs(o[0, 0, i, c] - want) < 1e-12
+            assert abs(lse[0, 0, i] - (mx + math.log(tot))) < 1e-12
+
+
+@pytest.mark.parametrize("causal,window", MODES)
+def test_decode_rows_are_the_last_rows_of_the_full_problem(causal, window):
+    """The Nq newest queries against all Nk keys give exactly the last Nq rows
+    of the Nk x Nk problem, whatever the earlier queries are."""
+    b, h, hkv, nk, nq, d = 2, 4, 2, 37, 5, 6
+    k, v = (_rand((b, hkv, nk, d), s) for s in (143, 144))
+    q_full = _rand((b, h, nk, d), 145)
+    o_full, l_full = ref.forward(q_full, k, v, 0.45, causal, window)
+    o, lse = ref.forward(q_full[:, :, nk - nq:], k, v, 0.45, causal, window)
+    np.testing.assert_allclose(o, o_full[:, :, nk - nq:], atol=1e-14)
+    np.testing.assert_allclose(lse, l_full[:, :, nk - nq:], atol=1e-14)
+
+
+def test_single_newest_query_causal_sees_every_key():
+    k, v = (_rand((1, 2, 29, 4), s) for s in (146, 147))
+    q = _rand((1, 2, 1, 4), 148)
+    oc, lc = ref.forward(q, k, v, 0.5, True)
+    of, lf = ref.forward(q, k, v, 0.5, False)
+    np.testing.assert_allclose(oc, of, atol=1e-15)
+    np.testing.assert_allclose(lc, lf, atol=1e-15)
+
+
+def test_decode_rejects_more_queries_than_keys():
+    with pytest.raises(ValueError):
+        ref.forward(_rand((1, 1, 6, 2), 1), _rand((1, 1, 5, 2), 2), _rand((1, 1, 5, 2), 3), 1.0)
