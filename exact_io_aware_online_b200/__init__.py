@@ -15,7 +15,7 @@ import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
            "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "fwd_varlen", "bwd_varlen", "fwd_strided", "bwd_strided",
-           "LIB_PATH", "HEADER_PATH"]
+           "fwd_decode", "decode_splits", "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_varlen.restype = i
     L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
     L.fa_bwd_varlen.restype = i
+    L.fa_fwd_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, sz, i, vp]
+    L.fa_fwd_decode.restype = i
     L.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, vp]
     L.fa_fwd_strided.restype = i
     L.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
@@ -143,6 +145,33 @@ def fwd_splitkv(q, k, v, num_splits: int, scale: float | None = None, causal: bo
                                 B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), int(num_splits),
                                 ws.data_ptr(), ws.numel(), _dtype_code(q), _stream_ptr(q.device))
     _check(code, "fa_fwd_splitkv")
+    return o, l
+
+
+def decode_splits(B: int, H: int, Nq: int, Nk: int, sms: int = 148) -> int:
+    """Key chunks per query tile for fwd_decode(): enough CTAs for about two per
+    SM, at most 16 and at most one per 128-key tile."""
+    units = B * H * ((Nq + 255) // 256)
+    return max(1, min(16, (Nk + 127) // 128, -(-2 * sms // units)))
+
+
+def fwd_decode(q, k, v, num_splits: int | None = None, scale: float | None = None, causal: bool = False,
+               window: int = -1, out=None, lse=None, workspace=None):
+    """O, LSE for q [B,H,Nq,d] against k/v [B,Hkv,Nk,d], Nq <= Nk: the queries
+    are the newest Nq positions (see fa_fwd_decode in fa.h); bf16 only."""
+    import torch
+    B, H, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    S = decode_splits(B, H, Nq, Nk) if num_splits is None else int(num_splits)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = int(lib().fa_fwd_splitkv_workspace_size(B, H, Nq, d, S))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    code = lib().fa_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                               B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), int(window), S,
+                               ws.data_ptr(), ws.numel(), _dtype_code(q), _stream_ptr(q.device))
+    _check(code, "fa_fwd_decode")
     return o, l
 
 

@@ -248,6 +248,56 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   return launched();
 }
 
+// Fewer queries than keys (decode): Nq query rows at positions Nk - Nq + i
+// against Nk keys, always through the split-KV kernel and the merge.
+template <int D>
+fa_status fwd_decode_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                          int Nq, int Nk, float scale, int causal, int window, cudaStream_t st, int splits, void* ws) {
+  using C = fa::FwdCfg<D>;
+  CUtensorMap tq, tk, tv, to;
+  bool f4[4];
+  if (!make_tile_map(&tq, q, B, H, Nq, D, fa::contiguous_strides(H, Nq, D), &f4[0]) ||
+      !make_tile_map(&tk, k, B, Hkv, Nk, D, fa::contiguous_strides(Hkv, Nk, D), &f4[1]) ||
+      !make_tile_map(&tv, v, B, Hkv, Nk, D, fa::contiguous_strides(Hkv, Nk, D), &f4[2]) ||
+      !make_tile_map(&to, o, B, H, Nq, D, fa::contiguous_strides(H, Nq, D), &f4[3]))
+    return FA_ERR_CUDA;
+  if (!set_smem(fa::fwd_sm100_kernel<D, true, false, false, true>, C::kSmemBytes)) return FA_ERR_CUDA;
+  fa::FwdDecodeParams p{};
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = Nq;
+  p.g = H / Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.window = window;
+  p.npairs = (Nq + 255) / 256;
+  p.ntiles_kv = (Nk + 127) / 128;
+  p.nbt = p.ntiles_kv;
+  p.Nk = Nk;
+  p.qoff = Nk - Nq;
+  {  // heads per group: Q, O and the (shared) K, V of a group within ~64 MiB of L2
+    const double unit = static_cast<double>(D) * (4.0 * Nq + 4.0 * Nk / p.g);
+    p.group = std::min(B * H, static_cast<int>(std::max(1.0, std::floor((64.0 * 1024 * 1024) / unit))));
+    p.group = std::max(p.g, p.group / p.g * p.g);  // whole GQA groups
+    p.group = std::min(p.group, B * H);
+  }
+  p.splits = splits;
+  p.nq2 = p.npairs * 256;
+  p.part_o = static_cast<float*>(ws);
+  p.part_m = reinterpret_cast<float4*>(static_cast<uint8_t*>(ws) +
+                                       align256(static_cast<size_t>(splits) * B * H * p.nq2 * D * 4));
+  const unsigned grid = static_cast<unsigned>(p.npairs) * B * H * splits;
+  mark_start(st);
+  fa::fwd_sm100_kernel<D, true, false, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+  mark_stop(st);
+  if (launched() != FA_OK) return FA_ERR_CUDA;
+  const unsigned cgrid = static_cast<unsigned>(B * H) * ((Nq + 31) / 32);
+  fa::fwd_combine_kernel<D><<<cgrid, 256, 0, st>>>(static_cast<const fa::FwdParams&>(p), o);
+  return launched();
+}
+
 void set_simt_strides(fa::SimtParams& s, const Layouts& L) {
   s.sq = L.q;
   s.sk = L.k;
@@ -613,6 +663,25 @@ fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void
   const bool contig = same_layouts(L, C0, 8);
   return run_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, scale, causal, window, dtype, stream,
                  contig ? nullptr : &L, nullptr, 0, seqlens);
+}
+
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                        int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void* workspace,
+                        size_t ws_bytes, fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (Nq < 1 || Nk < Nq) return FA_ERR_INVALID_ARG;
+  fa_status s = check_common(B, H, Hkv, Nk, d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (num_splits < 1 || num_splits > fa::kMaxSplits) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  if (!workspace || ws_bytes < splitkv_ws_bytes(B, H, Nq, d, num_splits)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return d == 64 ? fwd_decode_bf16<64>(q, k, v, o, lse, B, H, Hkv, Nq, Nk, scale, causal, window, st, num_splits,
+                                       workspace)
+                 : fwd_decode_bf16<128>(q, k, v, o, lse, B, H, Hkv, Nq, Nk, scale, causal, window, st, num_splits,
+                                        workspace);
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype) {

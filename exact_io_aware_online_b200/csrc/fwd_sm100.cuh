@@ -68,8 +68,14 @@ struct FwdStridedParams : FwdParams {
   unsigned map4;
 };
 constexpr unsigned kMapQ = 1, kMapK = 2, kMapV = 4, kMapO = 8;
-template <bool kStrided>
-using FwdArgs = std::conditional_t<kStrided, FwdStridedParams, FwdParams>;
+// Arguments of the decode instantiation (split-KV only): N is the number of
+// query rows Nq, the keys number Nk >= Nq, and query row i sits at position
+// qoff + i with qoff = Nk - Nq (the newest Nq tokens of the sequence).
+struct FwdDecodeParams : FwdParams {
+  int Nk, qoff;
+};
+template <bool kStrided, bool kDecode = false>
+using FwdArgs = std::conditional_t<kDecode, FwdDecodeParams, std::conditional_t<kStrided, FwdStridedParams, FwdParams>>;
 
 // Partial-output layout: row n = 32 g + lane; the 16-byte unit u (columns
 // 4u..4u+3) of 32 consecutive rows is contiguous, so a warp whose lane owns a
@@ -135,11 +141,11 @@ __device__ __forceinline__ void exp_row_to_tmem(const float (&s)[128], float sl2
   lb += b0 + b1;
 }
 
-template <int D, bool kSplit, bool kMask, bool kStrided = false>
+template <int D, bool kSplit, bool kMask, bool kStrided = false, bool kDecode = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                     const FwdArgs<kStrided> p) {
+                     const FwdArgs<kStrided, kDecode> p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -176,13 +182,20 @@ __global__ void __launch_bounds__(384, 1)
   const int kvh = b * p.Hkv + h / p.g;
   const int q0 = pair * 256;
   const int Lb = p.seqlens ? max(0, min(p.seqlens[b], p.N)) : p.N;  // valid rows of this batch entry
+  // Valid keys and the position of query row 0 (decode: Nk keys, queries are
+  // the newest rows; otherwise the same rows as the queries, position 0).
+  int Lk = Lb, qoff = 0;
+  if constexpr (kDecode) {
+    Lk = p.Nk;
+    qoff = p.qoff;
+  }
   const int qlast = min(q0 + 255, Lb - 1);
   int jlo = 0, jhi = p.ntiles_kv - 1;
-  jhi = min(jhi, (max(Lb, 1) - 1) / 128);  // key tiles holding valid rows
-  if (p.causal) jhi = min(jhi, qlast / 128);
+  jhi = min(jhi, (max(Lk, 1) - 1) / 128);  // key tiles holding valid rows
+  if (p.causal) jhi = min(jhi, (qlast + qoff) / 128);
   if (p.window >= 0) {
-    jlo = max(0, q0 - p.window) / 128;
-    jhi = min(jhi, (qlast + p.window) / 128);
+    jlo = max(0, q0 + qoff - p.window) / 128;
+    jhi = min(jhi, (qlast + qoff + p.window) / 128);
   }
   if (kSplit) {  // my contiguous chunk of the key-tile range (possibly empty)
     const int chunk = (jhi - jlo + p.splits) / p.splits;
@@ -377,16 +390,17 @@ __global__ void __launch_bounds__(384, 1)
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sraw[c]);
-      bool full = kv0 + 127 < Lb && !block_off;
-      if (p.causal) full = full && (kv0 + 127 <= tq0);
-      if (p.window >= 0) full = full && (tq0 + 127 - kv0 <= p.window) && (kv0 + 127 - tq0 <= p.window);
+      const int tpos = tq0 + qoff, qpos = qrow + qoff;  // positions of the tile's first row and of my row
+      bool full = kv0 + 127 < Lk && !block_off;
+      if (p.causal) full = full && (kv0 + 127 <= tpos);
+      if (p.window >= 0) full = full && (tpos + 127 - kv0 <= p.window) && (kv0 + 127 - tpos <= p.window);
       if (!full) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
           const int key = kv0 + c;
-          bool keep = key < Lb && !block_off;
-          if (p.causal) keep = keep && key <= qrow;
-          if (p.window >= 0) keep = keep && abs(qrow - key) <= p.window;
+          bool keep = key < Lk && !block_off;
+          if (p.causal) keep = keep && key <= qpos;
+          if (p.window >= 0) keep = keep && abs(qpos - key) <= p.window;
           if (!keep) s[c] = -INFINITY;
         }
       }

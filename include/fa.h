@@ -95,6 +95,25 @@ fa_status fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, f
 size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits);
 
 /*
+ * Decode: Nq <= Nk queries against Nk keys, forward only.  q, o [B, H, Nq, d],
+ * k, v [B, Hkv, Nk, d], lse [B, H, Nq], all contiguous.  The queries are the
+ * newest Nq tokens of a length-Nk sequence: query row i sits at position
+ * Nk - Nq + i, and the causal / window predicate applies to that position
+ * ("FlashAttention" guide page, "Key takeaways": prefill and decode want
+ * different mappings of the same math).  With Nq == Nk this is fa_fwd.  The
+ * key range of every query tile is cut into num_splits chunks processed by
+ * separate CTAs, whose partial online-softmax states are merged on the device
+ * exactly as in fa_fwd_splitkv -- what keeps a single short query tile from
+ * running on one SM.  workspace: at least
+ * fa_fwd_splitkv_workspace_size(B, H, Nq, d, num_splits) bytes, 16-byte
+ * aligned.  bf16 only (FA_ERR_UNSUPPORTED otherwise); FA_ERR_INVALID_ARG for
+ * Nq < 1, Nk < Nq or num_splits outside [1, 16]; other errors as fa_fwd.
+ */
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                        int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void* workspace,
+                        size_t ws_bytes, fa_dtype dtype, void* stream);
+
+/*
  * Block-sparse forward and backward: as fa_fwd / fa_bwd with an extra 0/1 mask
  * over 128 x 128 blocks of the score matrix; a key is allowed only if the
  * causal / window predicate allows it AND its block is on.  Block sparsity is

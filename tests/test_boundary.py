@@ -21,7 +21,7 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_strided", "fa_bwd_strided"):
+              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_strided", "fa_bwd_strided", "fa_fwd_decode"):
         assert n in names
 
 
@@ -209,3 +209,31 @@ def test_strided_helper_requires_contiguous_last_axis():
         fa._strides_of(x)
     st = fa._strides_of(torch.zeros(2, 8, 3, 64).transpose(1, 2))
     assert (st[0].batch, st[0].head, st[0].row) == (8 * 3 * 64, 64, 3 * 64)
+
+
+def test_decode_rejects_bad_arguments(L):
+    f = ctypes.c_float(0.125)
+    need = L.fa_fwd_splitkv_workspace_size(2, 8, 3, 128, 4)
+
+    def call(**kw):
+        a = dict(q=A, B=2, H=8, Hkv=2, Nq=3, Nk=1000, d=128, splits=4, ws=need, dtype=0)
+        a.update(kw)
+        return L.fa_fwd_decode(a["q"], A, A, A, A, a["B"], a["H"], a["Hkv"], a["Nq"], a["Nk"], a["d"], f, 1, -1,
+                               a["splits"], A, a["ws"], a["dtype"], None)
+
+    assert call(q=None) == 1
+    assert call(Nq=0) == 1
+    assert call(Nq=1001) == 1                  # more queries than keys
+    assert call(splits=0) == 1 and call(splits=17) == 1
+    assert call(H=7) == 1                      # H % Hkv
+    assert call(d=96) == 2
+    assert call(dtype=1) == 2                  # bf16 only
+    assert call(q=A + 8) == 3
+    assert call(ws=need - 1) == 4
+
+
+def test_decode_split_heuristic():
+    assert fa.decode_splits(1, 32, 1, 32768) == 10      # 32 units -> ~2 CTAs per SM
+    assert fa.decode_splits(64, 32, 1, 32768) == 1
+    assert fa.decode_splits(1, 1, 1, 300) == 3          # at most one chunk per key tile
+    assert fa.decode_splits(1, 1, 1, 1 << 20) == 16
