@@ -394,6 +394,73 @@ def run_ours(args, w, world, rank, local):
     return 0
 
 
+DECODE_SHAPE = dict(B=8, H=32, Hkv=8, Nk=32768, d=128)  # one new token per sequence vs a 32768-token cache
+
+
+def run_decode(args, rank, local):
+    """Decode forward (fa_fwd_decode): Nq new queries against a long cache,
+    causal, bf16.  Memory-bound: the figure of merit is the bytes it must read
+    (K and V once, plus Q) and write (O, LSE) per second, against the measured
+    HBM copy bandwidth."""
+    import torch
+    import exact_io_aware_online_b200 as fa
+    from exact_io_aware_online_b200 import _build
+    if rank == 0:
+        _build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    S = DECODE_SHAPE
+    B, H, Hkv, Nk, d, Nq = S["B"], S["H"], S["Hkv"], S["Nk"], S["d"], args.decode
+    g = torch.Generator("cpu").manual_seed(90 + rank)
+    q = torch.randn((B, H, Nq, d), generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn((B, Hkv, Nk, d), generator=g).to(torch.bfloat16).to(dev)
+    splits = args.splits or fa.decode_splits(B, H, Hkv, Nq, Nk)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=dev)
+    ws = torch.empty(int(fa.lib().fa_fwd_decode_workspace_size(B, H, Hkv, Nq, d, splits)), dtype=torch.uint8,
+                     device=dev)
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in ev:
+        a.record()
+        b.record()
+    # the cache (2 x 512 MiB) is larger than L2, so every step reads it from HBM
+    for _ in range(args.warmup):
+        fa.fwd_decode(q, k, v, splits, 1.0 / d ** 0.5, True, out=o, lse=lse, workspace=ws)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t0.record(stream)
+        for i in range(K):
+            fa.set_timing_events(*ev[i])
+            fa.fwd_decode(q, k, v, splits, 1.0 / d ** 0.5, True, out=o, lse=lse, workspace=ws)
+        fa.set_timing_events(None, None)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if fa.device_status() != 0:
+        raise RuntimeError("device-side timeout during the timed region")
+    ms = t0.elapsed_time(t1) / K
+    kern = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    algo = (2 * B * Hkv * Nk * d + 2 * B * H * Nq * d) * 2 + B * H * Nq * 4  # K, V, Q read; O written; LSE
+    pk, src = peaks()
+    peak = float(pk["hbm_gbs"])
+    if rank == 0:
+        print(json.dumps({
+            "metric": "decode forward GB/s (bf16, causal, one cache read per step)", "value": algo / (ms * 1e-3) / 1e9,
+            "unit": "GB/s", "n_gpus": 1, "steps": K, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"decode_b{B}h{H}kv{Hkv}_nq{Nq}_nk{Nk}_d{d}", "splits": splits,
+                       "l2": "cache of 1 GiB, larger than L2 (no flush)"},
+            "roofline": {"bound": "hbm", "kernel": "fwd_sm100_kernel (decode, split)", "achieved":
+                         algo / (kern * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": algo / (kern * 1e-3) / 1e9 / peak, "traffic": None,
+                         "peak_kind": f"HBM copy ({src})", "kernel_ms": kern},
+            "clocks": clk.summary(), "gpu_launches": 2 * K}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -407,6 +474,9 @@ def main():
     ap.add_argument("--splits", type=int, default=0, help="split-KV forward with this many key chunks (0: off)")
     ap.add_argument("--block-density", type=float, default=None,
                     help="block-sparse attention with a seeded mask keeping this fraction of 128x128 blocks")
+    ap.add_argument("--decode", type=int, default=0,
+                    help="time the decode forward instead: this many new queries per sequence against a "
+                         "32768-token cache (B=8, 32 query heads on 8 kv heads, d=128, causal)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -415,6 +485,10 @@ def main():
     config_of.splits = args.splits
     config_of.block_density = args.block_density
     try:
+        if args.decode:
+            if world > 1 or args.impl != "ours":
+                raise SystemExit("--decode: one GPU, --impl ours only")
+            return run_decode(args, rank, local)
         if args.impl == "reference":
             return run_reference(args, w, world, rank)
         return run_ours(args, w, world, rank, local)

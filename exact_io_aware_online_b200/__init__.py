@@ -80,6 +80,8 @@ def lib() -> ctypes.CDLL:
     L.fa_bwd_varlen.restype = i
     L.fa_fwd_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, i, i, i, vp, sz, i, vp]
     L.fa_fwd_decode.restype = i
+    L.fa_fwd_decode_workspace_size.argtypes = [i, i, i, i, i, i]
+    L.fa_fwd_decode_workspace_size.restype = sz
     L.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, vp]
     L.fa_fwd_strided.restype = i
     L.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
@@ -148,11 +150,20 @@ def fwd_splitkv(q, k, v, num_splits: int, scale: float | None = None, causal: bo
     return o, l
 
 
-def decode_splits(B: int, H: int, Nq: int, Nk: int, sms: int = 148) -> int:
-    """Key chunks per query tile for fwd_decode(): enough CTAs for about two per
-    SM, at most 16 and at most one per 128-key tile."""
-    units = B * H * ((Nq + 255) // 256)
-    return max(1, min(16, (Nk + 127) // 128, -(-2 * sms // units)))
+def decode_splits(B: int, H: int, Hkv: int, Nq: int, Nk: int, sms: int = 148) -> int:
+    """Key chunks per query tile for fwd_decode().  The kernel runs one CTA per
+    (kv head, 256 packed query rows, chunk), all of about the same length, so
+    the count is chosen for whole waves over the SMs: the largest share of
+    busy SM slots in the last wave, at most 16 chunks and at most one per
+    128-key tile."""
+    units = B * Hkv * (((H // Hkv) * Nq + 255) // 256)
+    best, best_eff = 1, -1.0
+    for s in range(1, min(16, (Nk + 127) // 128) + 1):
+        ctas = units * s
+        eff = ctas / (sms * -(-ctas // sms))
+        if eff > best_eff + 1e-9:
+            best, best_eff = s, eff
+    return best
 
 
 def fwd_decode(q, k, v, num_splits: int | None = None, scale: float | None = None, causal: bool = False,
@@ -163,10 +174,10 @@ def fwd_decode(q, k, v, num_splits: int | None = None, scale: float | None = Non
     B, H, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
-    S = decode_splits(B, H, Nq, Nk) if num_splits is None else int(num_splits)
+    S = decode_splits(B, H, Hkv, Nq, Nk) if num_splits is None else int(num_splits)
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
-    need = int(lib().fa_fwd_splitkv_workspace_size(B, H, Nq, d, S))
+    need = int(lib().fa_fwd_decode_workspace_size(B, H, Hkv, Nq, d, S))
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
     code = lib().fa_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                                B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), int(window), S,

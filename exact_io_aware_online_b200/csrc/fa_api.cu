@@ -170,6 +170,12 @@ inline size_t splitkv_ws_bytes(int B, int H, int N, int d, int splits) {
          align256(static_cast<size_t>(splits) * B * H * nq2 * 16);
 }
 
+// Decode partials: the g query heads of a kv head form one virtual head of
+// g * Nq rows.
+inline size_t decode_ws_bytes(int B, int H, int Hkv, int Nq, int d, int splits) {
+  return splitkv_ws_bytes(B, Hkv, (H / Hkv) * Nq, d, splits);
+}
+
 // splits == 0: the plain forward; splits >= 1: split-KV partials into `ws`
 // followed by the merge kernel.  L: non-null for a layout other than the
 // contiguous one (then no splits and no block mask); those calls run the
@@ -249,51 +255,55 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
 }
 
 // Fewer queries than keys (decode): Nq query rows at positions Nk - Nq + i
-// against Nk keys, always through the split-KV kernel and the merge.
+// against Nk keys, always through the split-KV kernel and the merge.  The g
+// query heads of a kv head are adjacent in [B, H, Nq, d], so they are handed to
+// the kernel as one virtual head of g * Nq rows ([B, Hkv, g * Nq, d], the same
+// memory; likewise the logsumexp): each CTA then reads a K/V tile once for the
+// whole group instead of once per query head.
 template <int D>
 fa_status fwd_decode_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
                           int Nq, int Nk, float scale, int causal, int window, cudaStream_t st, int splits, void* ws) {
   using C = fa::FwdCfg<D>;
+  const int g = H / Hkv, Nv = g * Nq;  // rows of a virtual head
   CUtensorMap tq, tk, tv, to;
   bool f4[4];
-  if (!make_tile_map(&tq, q, B, H, Nq, D, fa::contiguous_strides(H, Nq, D), &f4[0]) ||
+  if (!make_tile_map(&tq, q, B, Hkv, Nv, D, fa::contiguous_strides(Hkv, Nv, D), &f4[0]) ||
       !make_tile_map(&tk, k, B, Hkv, Nk, D, fa::contiguous_strides(Hkv, Nk, D), &f4[1]) ||
       !make_tile_map(&tv, v, B, Hkv, Nk, D, fa::contiguous_strides(Hkv, Nk, D), &f4[2]) ||
-      !make_tile_map(&to, o, B, H, Nq, D, fa::contiguous_strides(H, Nq, D), &f4[3]))
+      !make_tile_map(&to, o, B, Hkv, Nv, D, fa::contiguous_strides(Hkv, Nv, D), &f4[3]))
     return FA_ERR_CUDA;
   if (!set_smem(fa::fwd_sm100_kernel<D, true, false, false, true>, C::kSmemBytes)) return FA_ERR_CUDA;
   fa::FwdDecodeParams p{};
   p.lse = lse;
   p.B = B;
-  p.H = H;
+  p.H = Hkv;
   p.Hkv = Hkv;
-  p.N = Nq;
-  p.g = H / Hkv;
+  p.N = Nv;
+  p.g = 1;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
   p.window = window;
-  p.npairs = (Nq + 255) / 256;
+  p.npairs = (Nv + 255) / 256;
   p.ntiles_kv = (Nk + 127) / 128;
   p.nbt = p.ntiles_kv;
   p.Nk = Nk;
   p.qoff = Nk - Nq;
-  {  // heads per group: Q, O and the (shared) K, V of a group within ~64 MiB of L2
-    const double unit = static_cast<double>(D) * (4.0 * Nq + 4.0 * Nk / p.g);
-    p.group = std::min(B * H, static_cast<int>(std::max(1.0, std::floor((64.0 * 1024 * 1024) / unit))));
-    p.group = std::max(p.g, p.group / p.g * p.g);  // whole GQA groups
-    p.group = std::min(p.group, B * H);
+  p.nq = Nq;
+  {  // virtual heads per group: their Q, O and K, V within ~64 MiB of L2
+    const double unit = static_cast<double>(D) * (4.0 * Nv + 4.0 * Nk);
+    p.group = std::min(B * Hkv, static_cast<int>(std::max(1.0, std::floor((64.0 * 1024 * 1024) / unit))));
   }
   p.splits = splits;
   p.nq2 = p.npairs * 256;
   p.part_o = static_cast<float*>(ws);
   p.part_m = reinterpret_cast<float4*>(static_cast<uint8_t*>(ws) +
-                                       align256(static_cast<size_t>(splits) * B * H * p.nq2 * D * 4));
-  const unsigned grid = static_cast<unsigned>(p.npairs) * B * H * splits;
+                                       align256(static_cast<size_t>(splits) * B * Hkv * p.nq2 * D * 4));
+  const unsigned grid = static_cast<unsigned>(p.npairs) * B * Hkv * splits;
   mark_start(st);
   fa::fwd_sm100_kernel<D, true, false, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
   mark_stop(st);
   if (launched() != FA_OK) return FA_ERR_CUDA;
-  const unsigned cgrid = static_cast<unsigned>(B * H) * ((Nq + 31) / 32);
+  const unsigned cgrid = static_cast<unsigned>(B * Hkv) * ((Nv + 31) / 32);
   fa::fwd_combine_kernel<D><<<cgrid, 256, 0, st>>>(static_cast<const fa::FwdParams&>(p), o);
   return launched();
 }
@@ -665,6 +675,12 @@ fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void
                  contig ? nullptr : &L, nullptr, 0, seqlens);
 }
 
+size_t fa_fwd_decode_workspace_size(int B, int H, int Hkv, int Nq, int d, int num_splits) {
+  if (Nq < 1 || check_common(B, H, Hkv, Nq, d, 1.0f, -1, FA_BF16) != FA_OK) return 0;
+  if (num_splits < 1 || num_splits > fa::kMaxSplits) return 0;
+  return decode_ws_bytes(B, H, Hkv, Nq, d, num_splits);
+}
+
 fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
                         int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void* workspace,
                         size_t ws_bytes, fa_dtype dtype, void* stream) {
@@ -675,7 +691,7 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
   if (num_splits < 1 || num_splits > fa::kMaxSplits) return FA_ERR_INVALID_ARG;
   if (dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
-  if (!workspace || ws_bytes < splitkv_ws_bytes(B, H, Nq, d, num_splits)) return FA_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < decode_ws_bytes(B, H, Hkv, Nq, d, num_splits)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? fwd_decode_bf16<64>(q, k, v, o, lse, B, H, Hkv, Nq, Nk, scale, causal, window, st, num_splits,

@@ -68,12 +68,26 @@ struct FwdStridedParams : FwdParams {
   unsigned map4;
 };
 constexpr unsigned kMapQ = 1, kMapK = 2, kMapV = 4, kMapO = 8;
-// Arguments of the decode instantiation (split-KV only): N is the number of
-// query rows Nq, the keys number Nk >= Nq, and query row i sits at position
-// qoff + i with qoff = Nk - Nq (the newest Nq tokens of the sequence).
+// Arguments of the decode instantiation (split-KV only).  The g query heads
+// that share a kv head are packed into one "virtual head" of g * nq rows (they
+// are adjacent in memory), so H = Hkv and g = 1 in the base fields and a CTA
+// reads each K/V tile once for the whole group.  Virtual row r is query
+// r % nq of its head, at position qoff + r % nq with qoff = Nk - nq (the
+// newest nq tokens of a length-Nk sequence).
 struct FwdDecodeParams : FwdParams {
-  int Nk, qoff;
+  int Nk, qoff, nq;
 };
+
+// Smallest and largest position of virtual rows r0..r1 (decode packing).
+__device__ __forceinline__ void decode_positions(int r0, int r1, int nq, int qoff, int& pmin, int& pmax) {
+  if (r1 - r0 + 1 >= nq || r0 % nq > r1 % nq) {  // every query position occurs
+    pmin = qoff;
+    pmax = qoff + nq - 1;
+  } else {
+    pmin = qoff + r0 % nq;
+    pmax = qoff + r1 % nq;
+  }
+}
 template <bool kStrided, bool kDecode = false>
 using FwdArgs = std::conditional_t<kDecode, FwdDecodeParams, std::conditional_t<kStrided, FwdStridedParams, FwdParams>>;
 
@@ -190,12 +204,14 @@ __global__ void __launch_bounds__(384, 1)
     qoff = p.qoff;
   }
   const int qlast = min(q0 + 255, Lb - 1);
+  int pmin = q0, pmax = qlast;  // positions of the pair's first and last valid rows
+  if constexpr (kDecode) decode_positions(q0, qlast, p.nq, qoff, pmin, pmax);
   int jlo = 0, jhi = p.ntiles_kv - 1;
   jhi = min(jhi, (max(Lk, 1) - 1) / 128);  // key tiles holding valid rows
-  if (p.causal) jhi = min(jhi, (qlast + qoff) / 128);
+  if (p.causal) jhi = min(jhi, pmax / 128);
   if (p.window >= 0) {
-    jlo = max(0, q0 + qoff - p.window) / 128;
-    jhi = min(jhi, (qlast + qoff + p.window) / 128);
+    jlo = max(0, pmin - p.window) / 128;
+    jhi = min(jhi, (pmax + p.window) / 128);
   }
   if (kSplit) {  // my contiguous chunk of the key-tile range (possibly empty)
     const int chunk = (jhi - jlo + p.splits) / p.splits;
@@ -365,6 +381,12 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY, l = 0.f, lb = 0.f;
     bool ok = true;
+    // positions: of my row, and the smallest / largest of the tile's rows
+    int qpos = qrow, tpmin = tq0, tpmax = tq0 + 127;
+    if constexpr (kDecode) {
+      qpos = qoff + qrow % p.nq;
+      decode_positions(tq0, max(tq0, min(tq0 + 127, Lb - 1)), p.nq, qoff, tpmin, tpmax);  // valid rows only
+    }
     int jcur = next_kv(jlo);
     for (int jj = 0; jj < nkv; ++jj, jcur = next_kv(jcur + 1)) {
       const int kv0 = jcur * 128;
@@ -390,10 +412,9 @@ __global__ void __launch_bounds__(384, 1)
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sraw[c]);
-      const int tpos = tq0 + qoff, qpos = qrow + qoff;  // positions of the tile's first row and of my row
       bool full = kv0 + 127 < Lk && !block_off;
-      if (p.causal) full = full && (kv0 + 127 <= tpos);
-      if (p.window >= 0) full = full && (tpos + 127 - kv0 <= p.window) && (kv0 + 127 - tpos <= p.window);
+      if (p.causal) full = full && (kv0 + 127 <= tpmin);
+      if (p.window >= 0) full = full && (tpmax - kv0 <= p.window) && (kv0 + 127 - tpmin <= p.window);
       if (!full) {
 #pragma unroll
         for (int c = 0; c < 128; ++c) {
@@ -458,11 +479,14 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
-          tmem_ld32(tO + c, o);
+          tmem_ld32(tO + c, o);  // warp-collective: every lane loads
           tmem_wait_ld();
+          if (n < Lb) {  // padding rows get weight 0 in the merge, which never reads their O~
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(dst + 32 * (c + 4 * u)) = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+            for (int u = 0; u < 8; ++u)
+              *reinterpret_cast<uint4*>(dst + 32 * (c + 4 * u)) =
+                  make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+          }
         }
         p.part_m[sbh * p.nq2 + n] = n < Lb ? make_float4(m_used, l, lb, 0.f) : make_float4(-INFINITY, 0.f, 0.f, 0.f);
       }

@@ -104,11 +104,14 @@ size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits)
  * key range of every query tile is cut into num_splits chunks processed by
  * separate CTAs, whose partial online-softmax states are merged on the device
  * exactly as in fa_fwd_splitkv -- what keeps a single short query tile from
- * running on one SM.  workspace: at least
- * fa_fwd_splitkv_workspace_size(B, H, Nq, d, num_splits) bytes, 16-byte
+ * running on one SM.  The H / Hkv query heads that share a kv head are
+ * processed together (their g * Nq rows are adjacent in q and o), so each K/V
+ * tile is read once per kv head, not once per query head.  workspace: at least
+ * fa_fwd_decode_workspace_size(B, H, Hkv, Nq, d, num_splits) bytes, 16-byte
  * aligned.  bf16 only (FA_ERR_UNSUPPORTED otherwise); FA_ERR_INVALID_ARG for
  * Nq < 1, Nk < Nq or num_splits outside [1, 16]; other errors as fa_fwd.
  */
+size_t fa_fwd_decode_workspace_size(int B, int H, int Hkv, int Nq, int d, int num_splits);
 fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
                         int Nq, int Nk, int d, float scale, int causal, int window, int num_splits, void* workspace,
                         size_t ws_bytes, fa_dtype dtype, void* stream);

@@ -213,7 +213,10 @@ def test_strided_helper_requires_contiguous_last_axis():
 
 def test_decode_rejects_bad_arguments(L):
     f = ctypes.c_float(0.125)
-    need = L.fa_fwd_splitkv_workspace_size(2, 8, 3, 128, 4)
+    need = L.fa_fwd_decode_workspace_size(2, 8, 2, 3, 128, 4)
+    assert need == L.fa_fwd_splitkv_workspace_size(2, 2, 12, 128, 4)  # 4 heads x 3 rows per kv head
+    assert L.fa_fwd_decode_workspace_size(2, 8, 2, 0, 128, 4) == 0
+    assert L.fa_fwd_decode_workspace_size(2, 8, 2, 3, 128, 17) == 0
 
     def call(**kw):
         a = dict(q=A, B=2, H=8, Hkv=2, Nq=3, Nk=1000, d=128, splits=4, ws=need, dtype=0)
@@ -233,7 +236,8 @@ def test_decode_rejects_bad_arguments(L):
 
 
 def test_decode_split_heuristic():
-    assert fa.decode_splits(1, 32, 1, 32768) == 10      # 32 units -> ~2 CTAs per SM
-    assert fa.decode_splits(64, 32, 1, 32768) == 1
-    assert fa.decode_splits(1, 1, 1, 300) == 3          # at most one chunk per key tile
-    assert fa.decode_splits(1, 1, 1, 1 << 20) == 16
+    # 64 units (B=8 x 8 kv heads, 4 x 1 packed rows each): 16 chunks fill 7 waves to 98.8%
+    assert fa.decode_splits(8, 32, 8, 1, 32768) == 16
+    assert fa.decode_splits(1, 1, 1, 1, 300) == 3          # at most one chunk per key tile
+    assert fa.decode_splits(37, 4, 1, 1, 1 << 20) == 4      # 37 x 4 = 148: one full wave
+    assert fa.decode_splits(148, 8, 8, 1, 32768) == 1

@@ -40,6 +40,8 @@ CASES = [
     ("full_noncausal_d64", 2, 2, 1, 17, 513, 64, False, -1, 5),
     ("causal_window_d128", 1, 2, 2, 40, 2048, 128, True, 200, 16),
     ("square_one_split", 1, 2, 1, 600, 600, 128, True, -1, 1),
+    ("packed_rows_span_pairs", 1, 8, 1, 70, 900, 64, True, 300, 2),   # 8 x 70 packed rows cross 256-row pairs
+    ("packed_window_d128", 2, 6, 2, 33, 1500, 128, False, 64, 4),
 ]
 
 
@@ -56,9 +58,10 @@ def test_decode_matches_oracle(case):
 
 
 def test_square_decode_equals_splitkv_bitwise():
-    """With Nq == Nk the decode instantiation does exactly what the split-KV
-    forward does."""
-    w = W.Workload("sq", 2, 4, 2, 900, 128, "bf16", True, -1, 72)
+    """With Nq == Nk and one query head per kv head (so the packing of query
+    heads is the identity) the decode instantiation does exactly what the
+    split-KV forward does."""
+    w = W.Workload("sq", 2, 4, 4, 900, 128, "bf16", True, -1, 72)
     x = {n: t.cuda() for n, t in W.make_inputs(w).items()}
     o1, l1 = fa.fwd_splitkv(x["q"], x["k"], x["v"], 3, w.scale, True)
     o2, l2 = fa.fwd_decode(x["q"], x["k"], x["v"], 3, w.scale, True)
