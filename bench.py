@@ -455,7 +455,8 @@ def run_decode(args, rank, local):
                        "l2": "cache of 1 GiB, larger than L2 (no flush)"},
             "roofline": {"bound": "hbm", "kernel": "fwd_sm100_kernel (decode, split)", "achieved":
                          algo / (kern * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
-                         "frac": algo / (kern * 1e-3) / 1e9 / peak, "traffic": None,
+                         "frac": algo / (kern * 1e-3) / 1e9 / peak,
+                         "traffic": ncu_traffic("fwd_sm100_kernel", f"decode_b{B}h{H}kv{Hkv}_nq{Nq}_nk{Nk}_d{d}"),
                          "peak_kind": f"HBM copy ({src})", "kernel_ms": kern},
             "clocks": clk.summary(), "gpu_launches": 2 * K}), flush=True)
     return 0

@@ -330,6 +330,9 @@ __global__ void __launch_bounds__(384, 1)
                   sdesc_sw128(aKV + slot * C::kTileBytes + k * 2048, 16384, 1024), kIdescO, acc || k > 0);
       };
       bool ok = nkv > 0 && mbar_wait(q_full, 0, abort_flag);
+      // decode: a second query tile of padding rows only gets no products
+      bool has1 = true;
+      if constexpr (kDecode) has1 = q0 + 128 < Lb;
       int it = 0;
       for (int jj = 0; ok && jj < nkv; ++jj, it += 2) {
         const int sK = it % C::kStages;
@@ -344,13 +347,17 @@ __global__ void __launch_bounds__(384, 1)
         qk(0, sK);
         umma_commit(&s_full[0]);
         if (jj > 0) {
-          if (!(ok = mbar_wait(&p_full[1], (jj - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          pv(1, sVprev, jj > 1);
+          if (has1) {
+            if (!(ok = mbar_wait(&p_full[1], (jj - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            pv(1, sVprev, jj > 1);
+          }
           umma_commit(&kv_empty[sVprev]);
         }
-        qk(1, sK);
-        umma_commit(&s_full[1]);
+        if (has1) {
+          qk(1, sK);
+          umma_commit(&s_full[1]);
+        }
         umma_commit(&kv_empty[sK]);
         const int sV = (it + 1) % C::kStages;
         if (!(ok = mbar_wait(&kv_full[sV], ((it + 1) / C::kStages) & 1, abort_flag))) break;
@@ -358,7 +365,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (ok) {
         const int sV = (it - 1) % C::kStages;
-        for (int t = 0; t < 2 && ok; ++t) {
+        for (int t = 0; t < (has1 ? 2 : 1) && ok; ++t) {
           if (!(ok = mbar_wait(&p_full[t], (nkv - 1) & 1, abort_flag))) break;
           tc_fence_after();
           pv(t, sV, nkv > 1);
@@ -387,8 +394,11 @@ __global__ void __launch_bounds__(384, 1)
       qpos = qoff + qrow % p.nq;
       decode_positions(tq0, max(tq0, min(tq0 + 127, Lb - 1)), p.nq, qoff, tpmin, tpmax);  // valid rows only
     }
+    int nkv_t = nkv;  // key tiles this query tile walks
+    if constexpr (kDecode)
+      if (t == 1 && q0 + 128 >= Lb) nkv_t = 0;  // padding rows only: no products were issued for them
     int jcur = next_kv(jlo);
-    for (int jj = 0; jj < nkv; ++jj, jcur = next_kv(jcur + 1)) {
+    for (int jj = 0; jj < nkv_t; ++jj, jcur = next_kv(jcur + 1)) {
       const int kv0 = jcur * 128;
       // block switched off for this query tile: every score of the tile is masked
       const bool block_off = kMask && !block_on(t, jcur);
@@ -471,7 +481,7 @@ __global__ void __launch_bounds__(384, 1)
       // ------------------------------------------------ partial results
       const int n = tq0 + r;  // < nq2 always
       const size_t sbh = static_cast<size_t>(split) * BH + bh;
-      if (nkv <= 0) {
+      if (nkv_t <= 0) {
         p.part_m[sbh * p.nq2 + n] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
       } else if (ok && (ok = mbar_wait(&o_full[t], 0, abort_flag))) {
         tc_fence_after();
