@@ -562,9 +562,10 @@ __global__ void __launch_bounds__(384, 1)
 // identity of "Flash attention and efficient attention" (Derivation, Step 3),
 // in base 2: m = max_s m_s, w_s = 2^(m_s - m),
 //   O = sum_s w_s O~_s / sum_s w_s lb_s,   LSE = (m + log2 sum_s w_s l_s) ln 2.
-// One block per (head, 32-row group): 32 threads compute the per-row weights,
-// all threads combine the 16-byte units (coalesced over rows), and the bf16
-// rows are written coalesced after a transpose through shared memory.
+// One block per (head, 32-row group): eight threads per row compute its
+// weights (two chunks each, combined by shuffles), all threads combine the
+// 16-byte units (coalesced over rows), and the bf16 rows are written coalesced
+// after a transpose through shared memory.
 constexpr int kMaxSplits = 16;
 
 template <int D>
@@ -575,21 +576,37 @@ __global__ void __launch_bounds__(256) fwd_combine_kernel(const FwdParams p, voi
   const int BH = p.B * p.H;
   const size_t bh = blockIdx.x / groups;
   const int g = static_cast<int>(blockIdx.x % groups);
-  if (threadIdx.x < 32) {
-    const int n = 32 * g + threadIdx.x;
+  {  // weights: eight threads per row, each over chunks j and j + 8, combined by shuffles
+    const int row = threadIdx.x >> 3, j = threadIdx.x & 7;
+    const int n = 32 * g + row;
+    float4 st[2];
     float m = -INFINITY;
-    for (int s = 0; s < p.splits; ++s) m = fmaxf(m, p.part_m[(static_cast<size_t>(s) * BH + bh) * p.nq2 + n].x);
-    float wl = 0.f, wlb = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      const float4 st = p.part_m[(static_cast<size_t>(s) * BH + bh) * p.nq2 + n];
-      const float w = (st.x == -INFINITY) ? 0.f : exp2f(st.x - m);
-      wgt[threadIdx.x][s] = w;
-      wl += w * st.y;
-      wlb += w * st.z;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int s = j + 8 * k;
+      st[k] = s < p.splits ? p.part_m[(static_cast<size_t>(s) * BH + bh) * p.nq2 + n]
+                           : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+      m = fmaxf(m, st[k].x);
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float w[2], wl = 0.f, wlb = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      w[k] = (st[k].x == -INFINITY) ? 0.f : exp2f(st[k].x - m);
+      wl += w[k] * st[k].y;
+      wlb += w[k] * st[k].z;
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      wl += __shfl_xor_sync(0xffffffffu, wl, o);
+      wlb += __shfl_xor_sync(0xffffffffu, wlb, o);
     }
     const float inv = wlb > 0.f ? 1.f / wlb : 0.f;
-    for (int s = 0; s < p.splits; ++s) wgt[threadIdx.x][s] *= inv;
-    if (n < p.N) p.lse[bh * p.N + n] = (wl > 0.f) ? (m + log2f(wl)) * kLn2 : -INFINITY;
+#pragma unroll
+    for (int k = 0; k < 2; ++k)
+      if (j + 8 * k < p.splits) wgt[row][j + 8 * k] = w[k] * inv;
+    if (j == 0 && n < p.N) p.lse[bh * p.N + n] = (wl > 0.f) ? (m + log2f(wl)) * kLn2 : -INFINITY;
   }
   __syncthreads();
 #pragma unroll
