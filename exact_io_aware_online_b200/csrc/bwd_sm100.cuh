@@ -113,45 +113,59 @@ struct BwdCfg {
 };
 
 // ---------------------------------------------------------------- preprocess
+// Half a warp per row (16 lanes x 16 bytes of O and of dO for D = 128, two rows
+// per warp instruction), four rows per warp, eight warps per block: wide
+// enough loads to keep HBM busy on this memory-bound pass.
+constexpr int kPreRowsPerWarp = 4;
+
 template <int D, bool kStrided = false>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p) {
+  constexpr int kLanesPerRow = D / 8;             // 8 bf16 (16 bytes) per lane
+  constexpr int kRowsPerPass = 32 / kLanesPerRow;  // 2 (D = 128) or 4 (D = 64)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t row = static_cast<size_t>(blockIdx.x) * 8 + warp;  // over B*H*Np
+  const int sub = lane / kLanesPerRow, part = lane % kLanesPerRow;
   const size_t rows = static_cast<size_t>(p.B) * p.H * p.Np;
-  if (row >= rows) return;
-  const size_t bh = row / p.Np;
-  const int n = static_cast<int>(row % p.Np);
-  float4* acc = reinterpret_cast<float4*>(p.dqacc + row * D);
-  for (int x = lane; x < D / 4; x += 32) acc[x] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (n >= valid_rows(p, static_cast<int>(bh / p.H))) {  // tile padding or a padded token
-    if (lane == 0) {
-      p.Drow[row] = 0.f;
-      p.lse2[row] = INFINITY;
-    }
-    return;
-  }
-  const __nv_bfloat162* o2;
-  const __nv_bfloat162* d2;
-  if constexpr (kStrided) {
-    const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
-    o2 = reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.o) + p.so.row(b, h, n));
-    d2 = reinterpret_cast<const __nv_bfloat162*>(static_cast<const __nv_bfloat16*>(p.dout) + p.sdo.row(b, h, n));
-  } else {
-    const size_t src = (bh * p.N + n) * D;
-    o2 = reinterpret_cast<const __nv_bfloat162*>(p.o) + src / 2;
-    d2 = reinterpret_cast<const __nv_bfloat162*>(p.dout) + src / 2;
-  }
-  float s = 0.f;
-  for (int x = lane; x < D / 2; x += 32) {
-    const float2 a = __bfloat1622float2(o2[x]);
-    const float2 c = __bfloat1622float2(d2[x]);
-    s = fmaf(a.x, c.x, fmaf(a.y, c.y, s));
-  }
+  const size_t row0 = (static_cast<size_t>(blockIdx.x) * 8 + warp) * kPreRowsPerWarp;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) {
-    p.Drow[row] = s;
-    p.lse2[row] = p.lse[bh * p.N + n] * 1.4426950408889634f;
+  for (int pass = 0; pass < kPreRowsPerWarp / kRowsPerPass; ++pass) {
+    const size_t row = row0 + pass * kRowsPerPass + sub;  // over B*H*Np
+    const bool in = row < rows;
+    const size_t bh = in ? row / p.Np : 0;
+    const int n = in ? static_cast<int>(row % p.Np) : 0;
+    if (in) {  // zero this row's slice of the dQ accumulator (row layout is irrelevant for zeros)
+      float4* acc = reinterpret_cast<float4*>(p.dqacc + row * D);
+      acc[2 * part] = make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[2 * part + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const bool valid = in && n < valid_rows(p, static_cast<int>(bh / p.H));
+    float s = 0.f;
+    if (valid) {
+      const __nv_bfloat16* orow;
+      const __nv_bfloat16* drow;
+      if constexpr (kStrided) {
+        const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
+        orow = static_cast<const __nv_bfloat16*>(p.o) + p.so.row(b, h, n);
+        drow = static_cast<const __nv_bfloat16*>(p.dout) + p.sdo.row(b, h, n);
+      } else {
+        orow = static_cast<const __nv_bfloat16*>(p.o) + (bh * p.N + n) * D;
+        drow = static_cast<const __nv_bfloat16*>(p.dout) + (bh * p.N + n) * D;
+      }
+      const uint4 a = reinterpret_cast<const uint4*>(orow)[part];
+      const uint4 c = reinterpret_cast<const uint4*>(drow)[part];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        s = fmaf(__uint_as_float(av[e] << 16), __uint_as_float(cv[e] << 16), s);
+        s = fmaf(__uint_as_float(av[e] & 0xffff0000u), __uint_as_float(cv[e] & 0xffff0000u), s);
+      }
+    }
+#pragma unroll
+    for (int off = kLanesPerRow / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (in && part == 0) {
+      // tile padding or a padded token: D = 0 and LSE = +inf, so its P is exactly 0
+      p.Drow[row] = valid ? s : 0.f;
+      p.lse2[row] = valid ? p.lse[bh * p.N + n] * 1.4426950408889634f : INFINITY;
+    }
   }
 }
 

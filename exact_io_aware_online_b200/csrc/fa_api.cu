@@ -409,7 +409,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
       !set_smem(fa::bwd_sm100_kernel<D, false, true>, C::kSmemBytes))
     return FA_ERR_CUDA;
   const size_t rows = static_cast<size_t>(B) * H * p.Np;
-  const unsigned pre_grid = static_cast<unsigned>((rows + 7) / 8);
+  const unsigned pre_grid = static_cast<unsigned>((rows + 8 * fa::kPreRowsPerWarp - 1) / (8 * fa::kPreRowsPerWarp));
   const unsigned grid = static_cast<unsigned>(p.ntiles) * B * Hkv;
   const unsigned dq_grid = static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32));
   if (L) {

@@ -5,6 +5,8 @@ Small cases cover every output element and span several tiles plus a ragged
 tail; the full-size workloads run in the launch configuration the benchmark
 times and are compared on whole sampled heads (whole GQA groups).
 """
+import time
+
 import pytest
 import torch
 
@@ -66,8 +68,11 @@ def test_fp32_workload_every_element():
     w = W.WORKLOADS["fp32_n256_d64"]
     x = W.make_inputs(w)
     got = gpu_run(w, x)
+    t0 = time.perf_counter()
     want = oracle_groups(w, x, _all_groups(w))
-    check_groups(w, got, want)
+    secs = time.perf_counter() - t0
+    worst = check_groups(w, got, want)
+    print("fp32_n256_d64", worst, f"oracle {secs:.2f} s (every head)")
 
 
 FULL = {
@@ -83,9 +88,11 @@ def test_full_workload_sampled_heads(name):
     w = W.WORKLOADS[name]
     x = W.make_inputs(w)
     got = gpu_run(w, x)
+    t0 = time.perf_counter()
     want = oracle_groups(w, x, FULL[name])
+    secs = time.perf_counter() - t0
     worst = check_groups(w, got, want)
-    print(name, worst)
+    print(name, worst, f"oracle {secs:.1f} s for {len(FULL[name])} kv group(s)")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
