@@ -206,6 +206,20 @@ def run_reference(args, w, world, rank):
 METRIC = "attention fwd+bwd TFLOP/s (bf16, causal N=8192 d=128) and % of BF16 tensor peak"
 
 
+def algorithmic_bytes(w: W.Workload, kind: str) -> float:
+    """Bytes a kernel must move between HBM and the SMs at the least: the
+    forward reads Q, K, V and writes O and the logsumexp; the backward kernel
+    reads Q, K, V, dO, the logsumexp and D, writes dK and dV, and moves the fp32
+    dQ accumulator in and out once."""
+    e = 2 if w.dtype == "bf16" else 4
+    q = w.B * w.H * w.N * w.d * e
+    kv = w.B * w.Hkv * w.N * w.d * e
+    rows = w.B * w.H * w.N
+    if kind == "fwd":
+        return q + 2 * kv + q + 4 * rows
+    return q + 2 * kv + q + 8 * rows + 2 * kv + 8 * rows * w.d
+
+
 def config_of(w: W.Workload, world: int):
     in_bytes = (2 * w.B * w.H + 2 * w.B * w.Hkv) * w.N * w.d * (2 if w.dtype == "bf16" else 4)
     return {"workload": w.name, "B": w.B, "H": w.H, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
@@ -326,13 +340,22 @@ def run_ours(args, w, world, rank, local):
         dom_name = dom_name.replace("sm100", "simt_f32")
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     peak = float(pk["bf16_tflops_sustained"])
-    roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": achieved / peak, "traffic": ncu_traffic(dom_name, w.name),
-            "peak_kind": f"bf16 dense, sustained ({src})",
-            "frac_of_burst_peak": achieved / float(pk["bf16_tflops"]),
-            "fwd_kernel_ms": fwd_k, "bwd_kernel_ms": bwd_k,
-            "fwd_kernel_tflops": fwd_f / (fwd_k * 1e-3) / 1e12,
-            "bwd_kernel_tflops": bwd_f / (bwd_k * 1e-3) / 1e12}
+    dom_bytes = algorithmic_bytes(w, "bwd" if dom_name.startswith("bwd") else "fwd")
+    ridge = peak * 1e12 / (float(pk["hbm_gbs"]) * 1e9)  # flop per byte where the two roofs meet
+    if dom_flops / dom_bytes >= ridge:
+        roof = {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_kind": f"bf16 dense, sustained ({src})",
+                "frac_of_burst_peak": achieved / float(pk["bf16_tflops"])}
+    else:  # below the ridge (narrow bands): the bytes that must move bound the kernel
+        gbs = dom_bytes / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom_name, "achieved": gbs, "peak": float(pk["hbm_gbs"]), "unit": "GB/s",
+                "frac": gbs / float(pk["hbm_gbs"]), "peak_kind": f"HBM copy ({src})",
+                "tensor_tflops": achieved, "tensor_frac_of_sustained": achieved / peak}
+    roof.update({"traffic": ncu_traffic(dom_name, w.name), "algorithmic_bytes": dom_bytes,
+                 "arithmetic_intensity": dom_flops / dom_bytes, "ridge": ridge,
+                 "fwd_kernel_ms": fwd_k, "bwd_kernel_ms": bwd_k,
+                 "fwd_kernel_tflops": fwd_f / (fwd_k * 1e-3) / 1e12,
+                 "bwd_kernel_tflops": bwd_f / (bwd_k * 1e-3) / 1e12})
 
     # ---- end to end: pinned host inputs -> device, fwd+bwd, results -> pinned host
     e2e = None
