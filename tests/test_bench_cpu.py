@@ -46,3 +46,26 @@ def test_gpu_arm_flags_are_validated():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "1"], capture_output=True,
                          text=True, timeout=120, cwd=ROOT)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def test_algorithmic_bytes_and_ridge_side():
+    """The byte model behind the roofline entry, written out for the headline
+    (bf16 B=2 H=16 N=8192 d=128): the forward moves Q, K, V in and O, LSE out;
+    the backward kernel moves Q, K, V, dO, LSE, D in, dK, dV out and the fp32
+    dQ accumulator in and out once.  The headline sits far above the ridge of
+    the measured peaks, the narrow-band window workload below it."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from exact_io_aware_online_b200 import workloads as W
+    w = W.WORKLOADS["bf16_causal_b2h16_n8192_d128"]
+    t = 2 * 16 * 8192 * 128 * 2  # one bf16 [B, H, N, d] tensor
+    rows = 2 * 16 * 8192
+    assert bench.algorithmic_bytes(w, "fwd") == 4 * t + 4 * rows
+    assert bench.algorithmic_bytes(w, "bwd") == 6 * t + 8 * rows + 8 * rows * 128
+    pk, _ = bench.peaks()
+    ridge = pk["bf16_tflops_sustained"] * 1e12 / (pk["hbm_gbs"] * 1e9)
+    f, b = W.flops(w)
+    assert b / bench.algorithmic_bytes(w, "bwd") > 5 * ridge
+    win = W.WORKLOADS["bf16_window128_h16_n32768_d64"]
+    fw, bw = W.flops(win)
+    assert bw / bench.algorithmic_bytes(win, "bwd") < ridge
