@@ -43,10 +43,18 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {  # the files each profiled kernel (and its launch configuration) is built from
+    "bwd_sm100_kernel": ("bwd_sm100.cuh", "sm100_ptx.cuh", "layout.cuh", "fa_api.cu"),
+    "fwd_sm100_kernel": ("fwd_sm100.cuh", "sm100_ptx.cuh", "layout.cuh", "fa_api.cu"),
+}
+
+
+def kernel_source_hash(kernel: str | None = None) -> str:
+    """Hash of the sources of `kernel` (of every CUDA source when None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_online_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KERNEL_SOURCES.get(kernel) if kernel else None
+    for name in sorted(names or os.listdir(csrc)):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -62,7 +70,7 @@ def ncu_traffic(kernel: str, workload: str):
     with open(p) as f:
         d = json.load(f)
     e = d.get(f"{kernel}@{workload}")
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e or e.get("source_hash") != kernel_source_hash(kernel):
         return None
     return e.get("bytes_per_launch")
 

@@ -613,16 +613,24 @@ __global__ void __launch_bounds__(256) fwd_combine_kernel(const FwdParams p, voi
   for (int k = 0; k < D / 32; ++k) {  // 32 rows x D/4 units, 256 threads
     const int f = threadIdx.x + 256 * k;
     const int u = f >> 5, l = f & 31;
+    // all chunks' loads issued before the sums (independent, one latency)
+    float4 a[kMaxSplits];
+    float wv[kMaxSplits];
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+      wv[s] = s < p.splits ? wgt[l][s] : 0.f;
+      a[s] = wv[s] != 0.f  // empty chunk or no allowed key: O~ unused
+                 ? *reinterpret_cast<const float4*>(
+                       p.part_o + fwd_part_unit<D>(static_cast<size_t>(s) * BH + bh, p.nq2, g, u) + 4 * l)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < p.splits; ++s) {
-      const float w = wgt[l][s];
-      if (w == 0.f) continue;  // empty chunk or no allowed key: O~ unused
-      const float4 a = *reinterpret_cast<const float4*>(
-          p.part_o + fwd_part_unit<D>(static_cast<size_t>(s) * BH + bh, p.nq2, g, u) + 4 * l);
-      acc.x = fmaf(w, a.x, acc.x);
-      acc.y = fmaf(w, a.y, acc.y);
-      acc.z = fmaf(w, a.z, acc.z);
-      acc.w = fmaf(w, a.w, acc.w);
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+      acc.x = fmaf(wv[s], a[s].x, acc.x);
+      acc.y = fmaf(wv[s], a[s].y, acc.y);
+      acc.z = fmaf(wv[s], a[s].z, acc.z);
+      acc.w = fmaf(wv[s], a[s].w, acc.w);
     }
     *reinterpret_cast<float4*>(&tile[l][4 * u]) = acc;
   }
