@@ -15,7 +15,7 @@ import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
            "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "fwd_varlen", "bwd_varlen", "fwd_strided", "bwd_strided",
-           "fwd_decode", "decode_splits", "LIB_PATH", "HEADER_PATH"]
+           "fwd_decode", "decode_splits", "fwd_packed", "bwd_packed", "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -82,6 +82,12 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_decode.restype = i
     L.fa_fwd_decode_workspace_size.argtypes = [i, i, i, i, i, i]
     L.fa_fwd_decode_workspace_size.restype = sz
+    L.fa_fwd_packed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, i, vp]
+    L.fa_fwd_packed.restype = i
+    L.fa_bwd_packed_workspace_size.argtypes = [vp, i, i, i, i]
+    L.fa_bwd_packed_workspace_size.restype = sz
+    L.fa_bwd_packed.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, i, i, vp]
+    L.fa_bwd_packed.restype = i
     L.fa_fwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, i, vp]
     L.fa_fwd_strided.restype = i
     L.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
@@ -369,6 +375,51 @@ def bwd_strided(q, k, v, o, lse, do, scale: float | None = None, causal: bool = 
                                 ws.data_ptr(), ws.numel(), B, H, Hkv, N, d, float(scale), int(bool(causal)),
                                 int(window), sp, code_t, _stream_ptr(q.device))
     _check(code, "fa_bwd_strided")
+    return dq, dk, dv
+
+
+def _host_offsets(cu_seqlens):
+    """ctypes int32 array of the B + 1 offsets (kept alive by the caller)."""
+    vals = [int(x) for x in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    return (ctypes.c_int * len(vals))(*vals), len(vals) - 1
+
+
+def fwd_packed(q, k, v, cu_seqlens, scale: float | None = None, causal: bool = False, window: int = -1,
+               out=None, lse=None):
+    """O [T,H,d] and LSE (flat: sequence b's [H, len_b] block at H * cu[b]) for
+    sequences packed along the token axis: q [T,H,d], k/v [T,Hkv,d], cu_seqlens
+    the B + 1 offsets (list or CPU tensor)."""
+    import torch
+    T, H, d = q.shape
+    Hkv = k.shape[1]
+    cu, B = _host_offsets(cu_seqlens)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty(T * H, dtype=torch.float32, device=q.device) if lse is None else lse
+    code = lib().fa_fwd_packed(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), cu,
+                               B, H, Hkv, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
+                               _stream_ptr(q.device))
+    _check(code, "fa_fwd_packed")
+    return o, l
+
+
+def bwd_packed(q, k, v, o, lse, do, cu_seqlens, scale: float | None = None, causal: bool = False, window: int = -1,
+               workspace=None, grads=None):
+    """bwd() of fwd_packed()."""
+    import torch
+    T, H, d = q.shape
+    Hkv = k.shape[1]
+    cu, B = _host_offsets(cu_seqlens)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    code_t = _dtype_code(q)
+    need = int(lib().fa_bwd_packed_workspace_size(cu, B, H, d, code_t))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    code = lib().fa_bwd_packed(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu, ws.data_ptr(), ws.numel(),
+                               B, H, Hkv, d, float(scale), int(bool(causal)), int(window), code_t,
+                               _stream_ptr(q.device))
+    _check(code, "fa_bwd_packed")
     return dq, dk, dv
 
 

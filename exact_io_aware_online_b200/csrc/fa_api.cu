@@ -478,6 +478,36 @@ fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, co
   return launched();
 }
 
+// ---------------------------------------------------------------- packed variable lengths
+// Sequence b is a one-entry problem of len_b = cu[b+1] - cu[b] rows whose
+// tensors start at token row cu[b] of the packed buffers (rows H*d elements
+// apart, heads d apart): each runs through the strided path with its own tensor
+// maps, so loads stop and stores clip at the sequence end.
+fa_status packed_lengths(const int* cu, int B, int* max_len) {
+  if (!cu || B < 1 || cu[0] != 0) return FA_ERR_INVALID_ARG;
+  int m = 0;
+  for (int b = 0; b < B; ++b) {
+    if (cu[b + 1] < cu[b]) return FA_ERR_INVALID_ARG;
+    m = std::max(m, cu[b + 1] - cu[b]);
+  }
+  *max_len = m;
+  return FA_OK;
+}
+
+// Layouts of sequence b: q, o, dout, dq [len, H, d]; k, v, dk, dv [len, Hkv, d].
+fa_status packed_layouts(int H, int Hkv, int len, int d, int es, Layouts* L) {
+  const fa::Strides qs{static_cast<long long>(len) * H * d, d, static_cast<long long>(H) * d};
+  const fa::Strides ks{static_cast<long long>(len) * Hkv * d, d, static_cast<long long>(Hkv) * d};
+  const fa::Strides in[8] = {qs, ks, ks, qs, qs, qs, ks, ks};
+  fa::Strides* out[8] = {&L->q, &L->k, &L->v, &L->o, &L->dout, &L->dq, &L->dk, &L->dv};
+  const int heads[8] = {H, Hkv, Hkv, H, H, H, Hkv, Hkv};
+  for (int t = 0; t < 8; ++t) {
+    const fa_status s = check_strides(in[t], 1, heads[t], len, d, es, t == 3 || t >= 5, out[t]);
+    if (s != FA_OK) return s;
+  }
+  return FA_OK;
+}
+
 // dtype / head-dimension dispatch shared by every entry point (arguments
 // already checked).
 fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
@@ -698,6 +728,70 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
                                        workspace)
                  : fwd_decode_bf16<128>(q, k, v, o, lse, B, H, Hkv, Nq, Nk, scale, causal, window, st, num_splits,
                                         workspace);
+}
+
+fa_status fa_fwd_packed(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                        int B, int H, int Hkv, int d, float scale, int causal, int window, fa_dtype dtype,
+                        void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int max_len = 0;
+  fa_status s = packed_lengths(cu_seqlens, B, &max_len);
+  if (s != FA_OK) return s;
+  s = check_common(1, H, Hkv, std::max(max_len, 1), d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
+  const size_t es = dtype == FA_BF16 ? 2 : 4;
+  for (int b = 0; b < B; ++b) {
+    const int len = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (len == 0) continue;
+    Layouts L{};
+    if ((s = packed_layouts(H, Hkv, len, d, static_cast<int>(es), &L)) != FA_OK) return s;
+    const size_t row = static_cast<size_t>(cu_seqlens[b]);
+    const size_t oq = row * H * d * es, ok = row * Hkv * d * es;
+    s = run_fwd(static_cast<const uint8_t*>(q) + oq, static_cast<const uint8_t*>(k) + ok,
+                static_cast<const uint8_t*>(v) + ok, static_cast<uint8_t*>(o) + oq, lse + row * H, 1, H, Hkv, len, d,
+                scale, causal, window, dtype, stream, H == 1 && Hkv == 1 ? nullptr : &L);
+    if (s != FA_OK) return s;
+  }
+  return FA_OK;
+}
+
+size_t fa_bwd_packed_workspace_size(const int* cu_seqlens, int B, int H, int d, fa_dtype dtype) {
+  int max_len = 0;
+  if (packed_lengths(cu_seqlens, B, &max_len) != FA_OK) return 0;
+  if (check_common(1, H, 1, std::max(max_len, 1), d, 1.0f, -1, dtype) != FA_OK) return 0;
+  return ws_layout(1, H, std::max(max_len, 1), d, dtype).total;
+}
+
+fa_status fa_bwd_packed(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens, void* workspace,
+                        size_t ws_bytes, int B, int H, int Hkv, int d, float scale, int causal, int window,
+                        fa_dtype dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int max_len = 0;
+  fa_status s = packed_lengths(cu_seqlens, B, &max_len);
+  if (s != FA_OK) return s;
+  s = check_common(1, H, Hkv, std::max(max_len, 1), d, scale, window, dtype);
+  if (s != FA_OK) return s;
+  s = check_bwd_buffers(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, 1, H, std::max(max_len, 1), d,
+                        dtype);
+  if (s != FA_OK) return s;
+  const size_t es = dtype == FA_BF16 ? 2 : 4;
+  for (int b = 0; b < B; ++b) {  // in stream order: each sequence reuses the workspace after the previous one
+    const int len = cu_seqlens[b + 1] - cu_seqlens[b];
+    if (len == 0) continue;
+    Layouts L{};
+    if ((s = packed_layouts(H, Hkv, len, d, static_cast<int>(es), &L)) != FA_OK) return s;
+    const size_t row = static_cast<size_t>(cu_seqlens[b]);
+    const size_t oq = row * H * d * es, ok = row * Hkv * d * es;
+    s = run_bwd(static_cast<const uint8_t*>(q) + oq, static_cast<const uint8_t*>(k) + ok,
+                static_cast<const uint8_t*>(v) + ok, static_cast<const uint8_t*>(o) + oq,
+                static_cast<const uint8_t*>(dout) + oq, lse + row * H, static_cast<uint8_t*>(dq) + oq,
+                static_cast<uint8_t*>(dk) + ok, static_cast<uint8_t*>(dv) + ok, workspace, 1, H, Hkv, len, d, scale,
+                causal, window, dtype, stream, H == 1 && Hkv == 1 ? nullptr : &L);
+    if (s != FA_OK) return s;
+  }
+  return FA_OK;
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype) {

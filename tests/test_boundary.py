@@ -21,7 +21,7 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_strided", "fa_bwd_strided", "fa_fwd_decode"):
+              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_strided", "fa_bwd_strided", "fa_fwd_decode", "fa_fwd_packed", "fa_bwd_packed"):
         assert n in names
 
 
@@ -241,3 +241,27 @@ def test_decode_split_heuristic():
     assert fa.decode_splits(1, 1, 1, 1, 300) == 3          # at most one chunk per key tile
     assert fa.decode_splits(37, 4, 1, 1, 1 << 20) == 4      # 37 x 4 = 148: one full wave
     assert fa.decode_splits(148, 8, 8, 1, 32768) == 1
+
+
+def test_packed_rejects_bad_arguments(L):
+    f = ctypes.c_float(0.125)
+
+    def cu(*vals):
+        return (ctypes.c_int * len(vals))(*vals)
+
+    def fwd(offsets, B, **kw):
+        a = dict(q=A, H=4, Hkv=2, d=128, dtype=0)
+        a.update(kw)
+        return L.fa_fwd_packed(a["q"], A, A, A, A, offsets, B, a["H"], a["Hkv"], a["d"], f, 1, -1, a["dtype"], None)
+
+    assert fwd(None, 2) == 1
+    assert fwd(cu(1, 5, 9), 2) == 1          # first offset must be 0
+    assert fwd(cu(0, 9, 5), 2) == 1          # offsets must not decrease
+    assert fwd(cu(0, 5, 9), 0) == 1          # B >= 1
+    assert fwd(cu(0, 5, 9), 2, H=3) == 1     # H % Hkv
+    assert fwd(cu(0, 5, 9), 2, d=96) == 2
+    assert fwd(cu(0, 5, 9), 2, q=A + 8) == 3
+    need = L.fa_bwd_packed_workspace_size(cu(0, 300, 301, 1000), 3, 4, 128, 0)
+    assert need == L.fa_bwd_workspace_size(1, 4, 699, 128, 0)  # the longest sequence
+    assert L.fa_bwd_packed_workspace_size(cu(0, 5, 4), 2, 4, 128, 0) == 0
+    assert L.fa_bwd_packed(*([A] * 9), cu(0, 300, 301, 1000), A, need - 1, 3, 4, 2, 128, f, 1, -1, 0, None) == 4
