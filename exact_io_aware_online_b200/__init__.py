@@ -282,9 +282,9 @@ def bwd_blocksparse(q, k, v, o, lse, do, block_mask, scale: float | None = None,
 
 def _seqlens_ptr(seqlens, B):
     import torch
-    if seqlens.dtype != torch.int32 or seqlens.numel() != B or not seqlens.is_cuda:
-        raise TypeError("seqlens must be a CUDA int32 tensor of B values")
-    return seqlens.contiguous().data_ptr()
+    if seqlens.dtype != torch.int32 or seqlens.numel() != B or not seqlens.is_cuda or not seqlens.is_contiguous():
+        raise TypeError("seqlens must be a contiguous CUDA int32 tensor of B values")
+    return seqlens.data_ptr()  # the caller's tensor: no temporary copy whose memory could be reused
 
 
 def fwd_varlen(q, k, v, seqlens, scale: float | None = None, causal: bool = False, window: int = -1,

@@ -265,3 +265,14 @@ def test_packed_rejects_bad_arguments(L):
     assert need == L.fa_bwd_workspace_size(1, 4, 699, 128, 0)  # the longest sequence
     assert L.fa_bwd_packed_workspace_size(cu(0, 5, 4), 2, 4, 128, 0) == 0
     assert L.fa_bwd_packed(*([A] * 9), cu(0, 300, 301, 1000), A, need - 1, 3, 4, 2, 128, f, 1, -1, 0, None) == 4
+
+
+def test_seqlens_helper_rejects_copies():
+    """A non-contiguous or host seqlens tensor is rejected rather than copied
+    to a temporary whose memory the allocator could hand out again before the
+    kernel reads it."""
+    torch = pytest.importorskip("torch")
+    with pytest.raises(TypeError):
+        fa._seqlens_ptr(torch.zeros(4, dtype=torch.int32), 4)        # host memory
+    with pytest.raises(TypeError):
+        fa._seqlens_ptr(torch.zeros(4, dtype=torch.int64), 4)        # wrong dtype
