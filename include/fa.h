@@ -65,7 +65,8 @@ typedef enum fa_dtype { FA_BF16 = 0, FA_FP32 = 1 } fa_dtype;
  * The online-softmax recurrence (running max m, running sum l, rescaled
  * unnormalised accumulator) is the one of "Flash attention and efficient
  * attention", section "Derivation: Incremental Softmax", Steps 1-3, applied
- * block after block of keys ("This generalizes to any number of blocks").
+ * block after block of keys (the page states that the two-block merge extends
+ * to any number of blocks).
  * Writes o [B,H,N,d] and lse [B,H,N]; reads q, k, v.  Deterministic.
  */
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -79,8 +80,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
  * running maximum m, sums l (and l of the bf16-rounded weights), unnormalised
  * accumulator O~ -- in `workspace`; a second kernel merges them with the
  * block-merge identity of "Flash attention and efficient attention",
- * "Derivation: Incremental Softmax", Step 3 ("This generalizes to any number of
- * blocks").  More CTAs for the same work: for small B*H with long N.
+ * "Derivation: Incremental Softmax", Step 3, which the page extends to any
+ * number of blocks.  More CTAs for the same work: for small B*H with long N.
  * bf16 only (FA_ERR_UNSUPPORTED for FA_FP32); 1 <= num_splits <= 16
  * (FA_ERR_INVALID_ARG otherwise); workspace: caller-owned device memory of at
  * least fa_fwd_splitkv_workspace_size() bytes, 16-byte aligned, contents
@@ -99,8 +100,8 @@ size_t fa_fwd_splitkv_workspace_size(int B, int H, int N, int d, int num_splits)
  * k, v [B, Hkv, Nk, d], lse [B, H, Nq], all contiguous.  The queries are the
  * newest Nq tokens of a length-Nk sequence: query row i sits at position
  * Nk - Nq + i, and the causal / window predicate applies to that position
- * ("FlashAttention" guide page, "Key takeaways": prefill and decode want
- * different mappings of the same math).  With Nq == Nk this is fa_fwd.  The
+ * ("FlashAttention" guide page, "Key takeaways": generating tokens calls for
+ * its own kernel mapping of the same computation).  With Nq == Nk this is fa_fwd.  The
  * key range of every query tile is cut into num_splits chunks processed by
  * separate CTAs, whose partial online-softmax states are merged on the device
  * exactly as in fa_fwd_splitkv -- what keeps a single short query tile from
@@ -146,7 +147,7 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
  * Padded variable lengths: as fa_fwd / fa_bwd on the same [B, H, N, d]
  * (and [B, Hkv, N, d]) layouts, where batch entry b holds only seqlens[b] valid
  * tokens at the start of its rows ("FlashAttention" guide page, "Tiling through
- * SRAM": padding changes tiling details, not the rule).  Keys at positions >=
+ * SRAM": padding only alters how the tiles are laid out, not what is computed).  Keys at positions >=
  * seqlens[b] are never attended to; query rows >= seqlens[b] get O = 0,
  * LSE = -inf and zero dQ; key rows >= seqlens[b] get zero dK, dV.  Whatever the
  * padding rows hold has no effect.  seqlens: device pointer to B int32 values,
@@ -207,7 +208,7 @@ fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void
  *                    H * cu_seqlens[b]
  * Each sequence is its own attention problem (causal / window relative to its
  * first token; "FlashAttention" guide page, "Tiling through SRAM": padding and
- * lengths change tiling details, not the rule).  Every sequence runs as a
+ * lengths only alter how the tiles are laid out, not what is computed).  Every sequence runs as a
  * separate one-entry launch of the strided path on `stream` (the offsets are
  * read on the host), so very many short sequences pay one launch each; empty
  * sequences launch nothing.  fa_bwd_packed's workspace: at least

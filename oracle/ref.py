@@ -17,15 +17,16 @@ What it computes, and where each step is stated:
   equal to it in exact arithmetic (page "FlashAttention paper", section
   "Exact, not approximate").
 * Masks -- causal keeps keys j <= i ("FlashAttention" guide page, section
-  "Tiling through SRAM": causal masks change tiling, not the rule); the local
+  "Tiling through SRAM": a causal mask alters which tiles are visited, never the result of the rule); the local
   window keeps |i - j| <= w, which reproduces the N=6, w=3 matrix of the
   "Flash attention and efficient attention" page, worked example
   "Local Attention Window" (there w counts the token and one neighbour on each
   side, i.e. half-width 1 here).
 * Saved softmax metadata -- the per-row natural-log logsumexp of the scaled,
-  masked scores, LSE_i = m_i + ln(sum_j exp(S_ij - m_i)).  The pages only call
-  it "a little softmax metadata" ("FlashAttention" guide page, "Tiling through
-  SRAM"); this is the plainest reading.
+  masked scores, LSE_i = m_i + ln(sum_j exp(S_ij - m_i)).  The pages say only
+  that a small amount of per-row softmax state is kept for training
+  ("FlashAttention" guide page, "Tiling through SRAM"); this is the plainest
+  reading.
 * Backward -- the pages say only that S and P are recomputed from Q, K, V
   ("Flash attention and efficient attention", section "Backward Pass:
   Recomputation").  The formulas below are the textbook softmax Jacobian for
@@ -42,7 +43,7 @@ What it computes, and where each step is stated:
   shared), and a key is allowed only if the causal / window predicate holds
   AND M[i // 128][j // 128] = 1.
 * Padding / variable lengths -- "FlashAttention" guide page, "Tiling through
-  SRAM": padding changes tiling details, not the rule.  Reading: batch entry b
+  SRAM": padding only alters how the tiles are laid out, not what is computed.  Reading: batch entry b
   holds L_b <= N valid tokens at the start of its [N, d] rows; keys >= L_b are
   never attended to and padded query rows (>= L_b) give O = 0, LSE = -inf and
   zero gradients, i.e. each batch entry is the attention of its first L_b
@@ -51,7 +52,8 @@ What it computes, and where each step is stated:
   diagonal is always allowed; possible under a block mask) give O = 0,
   LSE = -inf and zero gradients.
 * Fewer queries than keys (decode) -- "FlashAttention" guide page, "Key
-  takeaways": prefill and decode change the mapping, not the math.  Reading:
+  takeaways": processing a whole prompt and generating one token at a time
+  call for different kernels that compute the same thing.  Reading:
   the Nq queries are the newest Nq tokens of a length-Nk sequence, so query i
   sits at position Nk - Nq + i and the causal / window predicate is applied to
   that position (forward only; Nq <= Nk).

@@ -399,8 +399,8 @@ def test_seqlens_equal_truncated_problems(causal, window):
 
 # --------------------------------------------------------------------------
 # Fewer queries than keys (decode): query i sits at position Nk - Nq + i
-# ("FlashAttention" guide page, "Key takeaways": decode changes the mapping,
-# not the math).
+# ("FlashAttention" guide page, "Key takeaways": generation needs its own kernel
+# mapping, with the same computation).
 # --------------------------------------------------------------------------
 def test_decode_brute_force_tiny():
     """Each query row written out with explicit loops: softmax over the keys its
