@@ -118,6 +118,63 @@ def _check(code: int, what: str):
         raise FAError(code, what)
 
 
+def _validate(like, *specs):
+    """Each (tensor, shape, name, contiguous) must have that shape, the dtype of
+    `like`, live on like's CUDA device and (unless the helper takes strided
+    layouts) be contiguous.  Shapes and dtypes are checked for all tensors
+    before placement.  The C entry points receive only pointers and sizes, so a
+    mismatch here would let a kernel read or write outside a buffer."""
+    for t, shape, name, _ in specs:
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if t.dtype != like.dtype:
+            raise TypeError(f"{name}: dtype {t.dtype}, expected {like.dtype}")
+    for t, _, name, contiguous in specs:
+        if not t.is_cuda or t.device != like.device:
+            raise ValueError(f"{name}: must be on the CUDA device of q, got {t.device} (q: {like.device})")
+        if contiguous and not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous (the *_strided helpers take other layouts)")
+
+
+def _same(t, shape, like, name: str, contiguous: bool = True):
+    _validate(like, (t, shape, name, contiguous))
+
+
+def _check_qkv(q, k, v, contiguous: bool = True, kv_rows=None, extra=()):
+    """q [B,H,N,d]; k, v [B,Hkv,kv_rows or N,d] of q's dtype and device, plus
+    the (tensor, shape, name) triples in `extra`."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [batch, heads, rows, head_dim]")
+    B, H, N, d = q.shape
+    Hkv = k.shape[1]
+    rows = N if kv_rows is None else kv_rows
+    specs = [(q, (B, H, N, d), "q"), (k, (B, Hkv, rows, d), "k"), (v, (B, Hkv, rows, d), "v"), *extra]
+    _validate(q, *[(t, sh, nm, contiguous) for t, sh, nm in specs])
+    return B, H, Hkv, N, d
+
+
+def _check_lse(lse, shape, q):
+    import torch
+    if lse.dtype != torch.float32 or tuple(lse.shape) != tuple(shape) or not lse.is_cuda or lse.device != q.device \
+            or not lse.is_contiguous():
+        raise ValueError(f"lse: must be a contiguous float32 tensor of shape {tuple(shape)} on {q.device}")
+
+
+def _bwd_specs(q, k, o, do, grads):
+    """(tensor, shape, name) triples of the backward's other tensors."""
+    specs = [(o, q.shape, "o"), (do, q.shape, "do")]
+    if grads is not None:
+        dq, dk, dv = grads
+        specs += [(dq, q.shape, "dq"), (dk, k.shape, "dk"), (dv, k.shape, "dv")]
+    return specs
+
+
+def _check_workspace(ws, device):
+    import torch
+    if ws.dtype != torch.uint8 or not ws.is_cuda or ws.device != device or not ws.is_contiguous():
+        raise ValueError("workspace: must be a contiguous torch.uint8 tensor on the inputs' device")
+
+
 def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype_code: int) -> int:
     return int(lib().fa_bwd_workspace_size(B, H, N, d, dtype_code))
 
@@ -125,8 +182,11 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int, dtype_code: int) -> int:
 def fwd(q, k, v, scale: float | None = None, causal: bool = False, window: int = -1, out=None, lse=None):
     """O, LSE = attention(q [B,H,N,d], k/v [B,Hkv,N,d]); outputs allocated if not given."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v)
+    if out is not None:
+        _same(out, q.shape, q, "out")
+    if lse is not None:
+        _check_lse(lse, (B, H, N), q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
@@ -142,8 +202,13 @@ def fwd_splitkv(q, k, v, num_splits: int, scale: float | None = None, causal: bo
     """fwd() with each query block's key range split into `num_splits` chunks
     (partials merged on the device); bf16 only."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v)
+    if out is not None:
+        _same(out, q.shape, q, "out")
+    if lse is not None:
+        _check_lse(lse, (B, H, N), q)
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
@@ -177,8 +242,16 @@ def fwd_decode(q, k, v, num_splits: int | None = None, scale: float | None = Non
     """O, LSE for q [B,H,Nq,d] against k/v [B,Hkv,Nk,d], Nq <= Nk: the queries
     are the newest Nq positions (see fa_fwd_decode in fa.h); bf16 only."""
     import torch
-    B, H, Nq, d = q.shape
-    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.dim() != 4:
+        raise ValueError("k must be 4-D [batch, kv heads, keys, head_dim]")
+    B, H, Hkv, Nq, d = _check_qkv(q, k, v, kv_rows=k.shape[2])
+    Nk = k.shape[2]
+    if out is not None:
+        _same(out, q.shape, q, "out")
+    if lse is not None:
+        _check_lse(lse, (B, H, Nq), q)
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     S = decode_splits(B, H, Hkv, Nq, Nk) if num_splits is None else int(num_splits)
     o = torch.empty_like(q) if out is None else out
@@ -196,8 +269,10 @@ def bwd(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, w
         workspace=None, grads=None):
     """dQ, dK, dV of sum(do * o); workspace and gradients allocated if not given."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v, extra=_bwd_specs(q, k, o, do, grads))
+    _check_lse(lse, (B, H, N), q)
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     code_t = _dtype_code(q)
     need = bwd_workspace_size(B, H, N, d, code_t)
@@ -217,8 +292,8 @@ def bwd_noalloc(q, k, v, o, lse, do, scale: float | None = None, causal: bool = 
     built-in scratch array replaces the workspace (see fa_bwd_noalloc in fa.h).
     Pass preallocated `grads`=(dq, dk, dv) to keep the call allocation-free."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v, extra=_bwd_specs(q, k, o, do, grads))
+    _check_lse(lse, (B, H, N), q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     code = lib().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
@@ -229,30 +304,33 @@ def bwd_noalloc(q, k, v, o, lse, do, scale: float | None = None, causal: bool = 
     return dq, dk, dv
 
 
-def _mask_args(block_mask, B, H):
+def _mask_args(block_mask, B, H, N, device):
     """(device pointer, head stride) for a uint8 block mask of shape [nb, nb]
-    (shared) or [B, H, nb, nb] (per query head)."""
+    (shared) or [B, H, nb, nb] (per query head), nb = ceil(N / 128)."""
     import torch
     if block_mask.dtype != torch.uint8 or not block_mask.is_contiguous():
         raise TypeError("block_mask must be a contiguous torch.uint8 tensor")
-    nb = block_mask.shape[-1]
-    if block_mask.dim() == 2:
-        return block_mask.data_ptr(), 0
-    if tuple(block_mask.shape) != (B, H, nb, nb):
-        raise ValueError("block_mask must be [nb, nb] or [B, H, nb, nb]")
-    return block_mask.data_ptr(), nb * nb
+    nb = (N + 127) // 128
+    if tuple(block_mask.shape) not in ((nb, nb), (B, H, nb, nb)):
+        raise ValueError(f"block_mask must be [{nb}, {nb}] or [{B}, {H}, {nb}, {nb}] for N = {N}")
+    if not block_mask.is_cuda or block_mask.device != device:
+        raise ValueError("block_mask must be on the CUDA device of q")
+    return block_mask.data_ptr(), (0 if block_mask.dim() == 2 else nb * nb)
 
 
 def fwd_blocksparse(q, k, v, block_mask, scale: float | None = None, causal: bool = False, window: int = -1,
                     out=None, lse=None):
     """fwd() restricted to the 128 x 128 blocks that `block_mask` switches on."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v)
+    if out is not None:
+        _same(out, q.shape, q, "out")
+    if lse is not None:
+        _check_lse(lse, (B, H, N), q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    mp, hs = _mask_args(block_mask, B, H)
+    mp, hs = _mask_args(block_mask, B, H, N, q.device)
     code = lib().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                                     B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), mp, hs,
                                     _dtype_code(q), _stream_ptr(q.device))
@@ -264,14 +342,16 @@ def bwd_blocksparse(q, k, v, o, lse, do, block_mask, scale: float | None = None,
                     window: int = -1, workspace=None, grads=None):
     """bwd() of fwd_blocksparse()."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v, extra=_bwd_specs(q, k, o, do, grads))
+    _check_lse(lse, (B, H, N), q)
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     code_t = _dtype_code(q)
     need = bwd_workspace_size(B, H, N, d, code_t)
     ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-    mp, hs = _mask_args(block_mask, B, H)
+    mp, hs = _mask_args(block_mask, B, H, N, q.device)
     code = lib().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                                     lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
                                     ws.numel(), B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), mp, hs,
@@ -291,8 +371,11 @@ def fwd_varlen(q, k, v, seqlens, scale: float | None = None, causal: bool = Fals
                out=None, lse=None):
     """fwd() where batch entry b holds seqlens[b] valid tokens (padded layout)."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v)
+    if out is not None:
+        _same(out, q.shape, q, "out")
+    if lse is not None:
+        _check_lse(lse, (B, H, N), q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
@@ -307,8 +390,10 @@ def bwd_varlen(q, k, v, o, lse, do, seqlens, scale: float | None = None, causal:
                workspace=None, grads=None):
     """bwd() of fwd_varlen()."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v, extra=_bwd_specs(q, k, o, do, grads))
+    _check_lse(lse, (B, H, N), q)
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     code_t = _dtype_code(q)
     need = bwd_workspace_size(B, H, N, d, code_t)
@@ -342,8 +427,11 @@ def fwd_strided(q, k, v, scale: float | None = None, causal: bool = False, windo
     (e.g. x.transpose(1, 2) of a [B,N,H,d] buffer).  O takes q's layout unless
     `out` is given; `seqlens` (optional) as in fwd_varlen()."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v, contiguous=False)
+    if out is not None:
+        _same(out, q.shape, q, "out", contiguous=False)
+    if lse is not None:
+        _check_lse(lse, (B, H, N), q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
@@ -361,8 +449,10 @@ def bwd_strided(q, k, v, o, lse, do, scale: float | None = None, causal: bool = 
     """bwd() of fwd_strided(); dq, dk, dv take the layouts of q, k, v unless
     `grads` is given."""
     import torch
-    B, H, N, d = q.shape
-    Hkv = k.shape[1]
+    B, H, Hkv, N, d = _check_qkv(q, k, v, contiguous=False, extra=_bwd_specs(q, k, o, do, grads))
+    _check_lse(lse, (B, H, N), q)
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     code_t = _dtype_code(q)
     need = bwd_workspace_size(B, H, N, d, code_t)
@@ -390,9 +480,18 @@ def fwd_packed(q, k, v, cu_seqlens, scale: float | None = None, causal: bool = F
     sequences packed along the token axis: q [T,H,d], k/v [T,Hkv,d], cu_seqlens
     the B + 1 offsets (list or CPU tensor)."""
     import torch
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q, k, v must be 3-D [tokens, heads, head_dim]")
     T, H, d = q.shape
     Hkv = k.shape[1]
     cu, B = _host_offsets(cu_seqlens)
+    if cu[B] != T:
+        raise ValueError(f"cu_seqlens[-1] = {cu[B]} but q holds {T} tokens")
+    _validate(q, (q, (T, H, d), "q", True), (k, (T, Hkv, d), "k", True), (v, (T, Hkv, d), "v", True))
+    if out is not None:
+        _same(out, q.shape, q, "out")
+    if lse is not None:
+        _check_lse(lse, (T * H,), q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty(T * H, dtype=torch.float32, device=q.device) if lse is None else lse
@@ -407,9 +506,19 @@ def bwd_packed(q, k, v, o, lse, do, cu_seqlens, scale: float | None = None, caus
                workspace=None, grads=None):
     """bwd() of fwd_packed()."""
     import torch
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("q, k, v must be 3-D [tokens, heads, head_dim]")
     T, H, d = q.shape
     Hkv = k.shape[1]
     cu, B = _host_offsets(cu_seqlens)
+    if cu[B] != T:
+        raise ValueError(f"cu_seqlens[-1] = {cu[B]} but q holds {T} tokens")
+    _validate(q, *[(t, sh, nm, True) for t, sh, nm in
+                   [(q, (T, H, d), "q"), (k, (T, Hkv, d), "k"), (v, (T, Hkv, d), "v"),
+                    *_bwd_specs(q, k, o, do, grads)]])
+    _check_lse(lse, (T * H,), q)
+    if workspace is not None:
+        _check_workspace(workspace, q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     code_t = _dtype_code(q)
     need = int(lib().fa_bwd_packed_workspace_size(cu, B, H, d, code_t))

@@ -276,3 +276,28 @@ def test_seqlens_helper_rejects_copies():
         fa._seqlens_ptr(torch.zeros(4, dtype=torch.int32), 4)        # host memory
     with pytest.raises(TypeError):
         fa._seqlens_ptr(torch.zeros(4, dtype=torch.int64), 4)        # wrong dtype
+
+
+def test_python_helpers_validate_before_the_c_layer():
+    """Sizes come from q alone, so every other tensor is checked against it
+    (shape, dtype, device, contiguity) before any pointer reaches the library."""
+    torch = pytest.importorskip("torch")
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        fa.fwd(q, torch.zeros(1, 1, 7, 64, dtype=torch.bfloat16), k)     # fewer key rows than q
+    with pytest.raises(ValueError, match="shape"):
+        fa.fwd(q, k, torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16))    # head dim mismatch
+    with pytest.raises(TypeError):
+        fa.fwd(q, k.float(), k)                                          # dtype mismatch
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.fwd(q, k, k)                                                  # host tensors never reach a kernel
+    with pytest.raises(ValueError, match="shape"):
+        fa.bwd(q, k, k, q, torch.zeros(1, 2, 8), torch.zeros(1, 2, 9, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="shape"):
+        fa.fwd_decode(q, torch.zeros(1, 1, 20, 64, dtype=torch.bfloat16), k)   # v rows differ from k
+    with pytest.raises(ValueError, match="tokens"):
+        fa.fwd_packed(torch.zeros(10, 2, 64, dtype=torch.bfloat16), torch.zeros(10, 1, 64, dtype=torch.bfloat16),
+                      torch.zeros(10, 1, 64, dtype=torch.bfloat16), [0, 4, 9])
+    with pytest.raises(ValueError):
+        fa._mask_args(torch.zeros(2, 2, dtype=torch.uint8), 1, 2, 300, torch.device("cpu"))  # 300 rows need 3 blocks
