@@ -1,7 +1,6 @@
 """GPU parity of fa_fwd_decode: Nq <= Nk queries, the newest Nq positions of
 the sequence, against the oracle's reading of the same (query i at position
 Nk - Nq + i), on seeded synthetic inputs."""
-import numpy as np
 import pytest
 import torch
 
