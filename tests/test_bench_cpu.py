@@ -69,3 +69,12 @@ def test_algorithmic_bytes_and_ridge_side():
     win = W.WORKLOADS["bf16_window128_h16_n32768_d64"]
     fw, bw = W.flops(win)
     assert bw / bench.algorithmic_bytes(win, "bwd") < ridge
+
+
+def test_bench_rejects_bad_option_combinations():
+    """Host-side option checks run before anything touches a GPU."""
+    for extra in (["--warmup", "2"], ["--decode", "1", "--impl", "reference"]):
+        out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *extra], capture_output=True,
+                             text=True, timeout=300, cwd=ROOT)
+        assert out.returncode != 0
+        assert "warmup" in out.stderr or "--decode" in out.stderr, out.stderr[-500:]
