@@ -15,7 +15,8 @@ import re
 
 __all__ = ["lib", "FAError", "FA_BF16", "FA_FP32", "fwd", "bwd", "bwd_workspace_size", "device_status",
            "exported_names", "set_timing_events", "bwd_noalloc", "fwd_splitkv", "fwd_blocksparse", "bwd_blocksparse", "fwd_varlen", "bwd_varlen", "fwd_strided", "bwd_strided",
-           "fwd_decode", "decode_splits", "fwd_packed", "bwd_packed", "LIB_PATH", "HEADER_PATH"]
+           "fwd_decode", "decode_splits", "fwd_packed", "bwd_packed", "debug_set_wait_limit", "debug_set_stall",
+           "LIB_PATH", "HEADER_PATH"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa.so")
@@ -92,6 +93,10 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_strided.restype = i
     L.fa_bwd_strided.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, i, f, i, i, vp, i, vp]
     L.fa_bwd_strided.restype = i
+    L.fa_debug_set_wait_limit.argtypes = [ctypes.c_ulonglong]
+    L.fa_debug_set_wait_limit.restype = i
+    L.fa_debug_set_stall.argtypes = [i]
+    L.fa_debug_set_stall.restype = i
     _lib = L
     return L
 
@@ -116,6 +121,15 @@ def _stream_ptr(device) -> int:
 def _check(code: int, what: str):
     if code != 0:
         raise FAError(code, what)
+
+
+def _on(device, fn, *args):
+    """Calls a library entry point with `device` current: the C ABI enqueues on
+    the stream it is given and rejects a stream of another device than the
+    current one."""
+    import torch
+    with torch.cuda.device(device):
+        return fn(*args)
 
 
 def _validate(like, *specs):
@@ -190,7 +204,7 @@ def fwd(q, k, v, scale: float | None = None, causal: bool = False, window: int =
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    code = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+    code = _on(q.device, lib().fa_fwd, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                         B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
                         _stream_ptr(q.device))
     _check(code, "fa_fwd")
@@ -214,7 +228,7 @@ def fwd_splitkv(q, k, v, num_splits: int, scale: float | None = None, causal: bo
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     need = int(lib().fa_fwd_splitkv_workspace_size(B, H, N, d, int(num_splits)))
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
-    code = lib().fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+    code = _on(q.device, lib().fa_fwd_splitkv, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                                 B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), int(num_splits),
                                 ws.data_ptr(), ws.numel(), _dtype_code(q), _stream_ptr(q.device))
     _check(code, "fa_fwd_splitkv")
@@ -258,7 +272,7 @@ def fwd_decode(q, k, v, num_splits: int | None = None, scale: float | None = Non
     l = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
     need = int(lib().fa_fwd_decode_workspace_size(B, H, Hkv, Nq, d, S))
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
-    code = lib().fa_fwd_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+    code = _on(q.device, lib().fa_fwd_decode, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                                B, H, Hkv, Nq, Nk, d, float(scale), int(bool(causal)), int(window), S,
                                ws.data_ptr(), ws.numel(), _dtype_code(q), _stream_ptr(q.device))
     _check(code, "fa_fwd_decode")
@@ -278,7 +292,7 @@ def bwd(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, w
     need = bwd_workspace_size(B, H, N, d, code_t)
     ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-    code = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+    code = _on(q.device, lib().fa_bwd, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
                         dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
                         B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), code_t,
                         _stream_ptr(q.device))
@@ -296,7 +310,7 @@ def bwd_noalloc(q, k, v, o, lse, do, scale: float | None = None, causal: bool = 
     _check_lse(lse, (B, H, N), q)
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-    code = lib().fa_bwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+    code = _on(q.device, lib().fa_bwd_noalloc, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                                 lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                                 B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
                                 _stream_ptr(q.device))
@@ -331,7 +345,7 @@ def fwd_blocksparse(q, k, v, block_mask, scale: float | None = None, causal: boo
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     mp, hs = _mask_args(block_mask, B, H, N, q.device)
-    code = lib().fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+    code = _on(q.device, lib().fa_fwd_blocksparse, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                                     B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), mp, hs,
                                     _dtype_code(q), _stream_ptr(q.device))
     _check(code, "fa_fwd_blocksparse")
@@ -352,7 +366,7 @@ def bwd_blocksparse(q, k, v, o, lse, do, block_mask, scale: float | None = None,
     ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     mp, hs = _mask_args(block_mask, B, H, N, q.device)
-    code = lib().fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+    code = _on(q.device, lib().fa_bwd_blocksparse, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                                     lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
                                     ws.numel(), B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window), mp, hs,
                                     code_t, _stream_ptr(q.device))
@@ -379,7 +393,7 @@ def fwd_varlen(q, k, v, seqlens, scale: float | None = None, causal: bool = Fals
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    code = lib().fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+    code = _on(q.device, lib().fa_fwd_varlen, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                                B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window),
                                _seqlens_ptr(seqlens, B), _dtype_code(q), _stream_ptr(q.device))
     _check(code, "fa_fwd_varlen")
@@ -399,7 +413,7 @@ def bwd_varlen(q, k, v, o, lse, do, seqlens, scale: float | None = None, causal:
     need = bwd_workspace_size(B, H, N, d, code_t)
     ws = torch.empty(need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-    code = lib().fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+    code = _on(q.device, lib().fa_bwd_varlen, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
                                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(),
                                B, H, Hkv, N, d, float(scale), int(bool(causal)), int(window),
                                _seqlens_ptr(seqlens, B), code_t, _stream_ptr(q.device))
@@ -437,7 +451,7 @@ def fwd_strided(q, k, v, scale: float | None = None, causal: bool = False, windo
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     st = _strides_of(q, k, v, o)
     sp = _seqlens_ptr(seqlens, B) if seqlens is not None else None
-    code = lib().fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+    code = _on(q.device, lib().fa_fwd_strided, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                                 ctypes.addressof(st), B, H, Hkv, N, d, float(scale), int(bool(causal)),
                                 int(window), sp, _dtype_code(q), _stream_ptr(q.device))
     _check(code, "fa_fwd_strided")
@@ -460,7 +474,7 @@ def bwd_strided(q, k, v, o, lse, do, scale: float | None = None, causal: bool = 
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     st = _strides_of(q, k, v, o, do, dq, dk, dv)
     sp = _seqlens_ptr(seqlens, B) if seqlens is not None else None
-    code = lib().fa_bwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+    code = _on(q.device, lib().fa_bwd_strided, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                                 lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ctypes.addressof(st),
                                 ws.data_ptr(), ws.numel(), B, H, Hkv, N, d, float(scale), int(bool(causal)),
                                 int(window), sp, code_t, _stream_ptr(q.device))
@@ -495,7 +509,7 @@ def fwd_packed(q, k, v, cu_seqlens, scale: float | None = None, causal: bool = F
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty(T * H, dtype=torch.float32, device=q.device) if lse is None else lse
-    code = lib().fa_fwd_packed(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), cu,
+    code = _on(q.device, lib().fa_fwd_packed, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), cu,
                                B, H, Hkv, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
                                _stream_ptr(q.device))
     _check(code, "fa_fwd_packed")
@@ -524,7 +538,7 @@ def bwd_packed(q, k, v, o, lse, do, cu_seqlens, scale: float | None = None, caus
     need = int(lib().fa_bwd_packed_workspace_size(cu, B, H, d, code_t))
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-    code = lib().fa_bwd_packed(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+    code = _on(q.device, lib().fa_bwd_packed, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
                                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu, ws.data_ptr(), ws.numel(),
                                B, H, Hkv, d, float(scale), int(bool(causal)), int(window), code_t,
                                _stream_ptr(q.device))
@@ -542,3 +556,13 @@ def device_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     import torch
     return int(lib().fa_last_device_status(torch.cuda.current_stream(device).cuda_stream))
+
+
+def debug_set_wait_limit(ns: int = 0):
+    """Test hook: limit (ns) of the kernels' waits on other roles; 0 restores the default."""
+    _check(lib().fa_debug_set_wait_limit(int(ns)), "fa_debug_set_wait_limit")
+
+
+def debug_set_stall(on: bool):
+    """Test hook: while on, the sm_100a kernels never issue their first tile load."""
+    _check(lib().fa_debug_set_stall(1 if on else 0), "fa_debug_set_stall")

@@ -9,8 +9,8 @@
 //   dK = scale dS^T Q,  dQ = scale dS K.
 //
 // Three kernels run on one stream:
-//   bwd_pre_kernel   D_i, LSE_i * log2(e) (+inf on padding rows) and a zeroed
-//                    fp32 dQ accumulator, all in the caller's workspace;
+//   bwd_pre_kernel   -D_i, -LSE_i * log2(e) (-inf on padding rows) and a
+//                    zeroed fp32 dQ accumulator, all in the caller's workspace;
 //   bwd_sm100_kernel one CTA per (batch, kv head, 128-key tile): K_j and V_j
 //                    stay in shared memory while the CTA walks every query
 //                    tile (of every query head of the GQA group) that can see
@@ -25,19 +25,25 @@
 //   warps 8-11  dQ drain (one thread per query row of the dQ tile) and the
 //               final dK/dV epilogue (one thread per key row)
 //   warp 12     tcgen05.mma issuer, stream A (S^T, dV) and TMEM owner
-//   warp 13     TMA producer (tiles of Q and dO, and the tile's LSE / D rows)
+//   warp 13     TMA producer of the Q tiles and their LSE / D rows
 //   warp 14     tcgen05.mma issuer, stream B (dP^T, dK, dQ)
-//   warp 15     idle (completes the fourth warpgroup)
+//   warp 15     TMA producer of the dO tiles
 // The two MMA streams touch disjoint TMEM regions (A: S^T and dV; B: dP^T, dK
 // and dQ), so each keeps its own order and a thread blocked pushing one
 // stream's instructions into a full tensor-core queue never delays the other.
 // Registers: 128 per thread at launch; the fourth warpgroup drops to 64, the
 // compute warpgroups rise to 144 and the drain to 160 (144 + 144 + 160 + 64 =
 // 4 * 128), so a drain thread holds a whole dQ row and releases the TMEM tile
-// before its reductions.
-// The dQ accumulator uses a lane-interleaved layout (see dqacc_index) so that
-// the drain's vector reductions are coalesced: one warp instruction adds 512
-// contiguous bytes instead of touching 32 rows.
+// at once.
+//
+// dQ reduction.  Every (key tile, query tile) pair adds a 128 x D fp32 partial
+// into the global accumulator.  The drain loads the partial from TMEM into
+// registers (freeing the TMEM tile), writes it to shared memory 32 columns at
+// a time and hands each 16 KB chunk to the TMA unit as one bulk reduce-add, so
+// the reductions never occupy the load/store queues that the compute warps
+// need for their shared-memory traffic.  The accumulator is laid out in the
+// same 16 KB chunks (see dqacc_chunk).
+//
 // The products are formed transposed (S^T = K Q^T, dP^T = V dO^T) so that P^T
 // and dS^T land in TMEM with one key row per lane and can be fed back, as
 // packed bf16, as the A operand of dV += P^T dO and dK += dS^T Q.  dS itself
@@ -61,9 +67,9 @@ struct BwdParams {
   const float* lse;  // [B*H*N] from the forward
   const void* o;     // bf16 [B*H*N*D]
   const void* dout;  // bf16 [B*H*N*D]
-  float* lse2;       // workspace [B*H*Np]: lse*log2(e), +inf on rows >= N
-  float* Drow;       // workspace [B*H*Np]: D_i, 0 on rows >= N
-  float* dqacc;      // workspace [B*H*Np*D]
+  float* nlse2;      // workspace [B*H*Np]: -lse*log2(e), -inf on rows >= N
+  float* nD;         // workspace [B*H*Np]: -D_i, 0 on rows >= N
+  float* dqacc;      // workspace [B*H*Np*D], in 16 KB chunks (dqacc_chunk)
   void* dq;          // bf16 [B*H*N*D]
   int B, H, Hkv, N, Np, g;
   float scale, scale_log2;
@@ -97,20 +103,26 @@ __device__ __forceinline__ int valid_rows(const BwdParams& p, int b) {
 template <int D>
 struct BwdCfg {
   static constexpr int kTileBytes = 128 * D * 2;
-  static constexpr int kChunks = D / 64;
-  static constexpr int kStages = (D == 128) ? 2 : 3;  // (Q, dO, LSE, D) tile sets in flight
+  static constexpr int kChunks = D / 64;                 // 64-column chunks of a bf16 tile
+  static constexpr int kQStages = (D == 128) ? 2 : 3;    // (Q, LSE, D) tile sets in flight
+  static constexpr int kDoStages = (D == 128) ? 1 : 2;   // dO tiles in flight
   static constexpr int kDsBytes = 128 * 128 * 2;
-  static constexpr int kVecBytes = 2 * 128 * 4;       // LSE*log2(e) and D of one query tile
-  static constexpr int kNumBars = 1 + 2 * kStages + 8;
+  static constexpr int kVecBytes = 2 * 128 * 4;          // -LSE*log2(e) and -D of one query tile
+  static constexpr int kDqChunkBytes = 128 * 32 * 4;     // 32 fp32 columns of a 128-row dQ tile
+  static constexpr int kDqChunks = D / 32;               // chunks per dQ tile
+  static constexpr int kDqStages = 2;                    // staging buffers of the dQ reduction
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDoStages + 11;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: at D = 128 this fits 227 KB exactly.
-  static constexpr int kSmemBytes =
-      2 * kTileBytes + kStages * 2 * kTileBytes + kDsBytes + kStages * kVecBytes + 8 * kNumBars + 16;
+  // so no alignment slack is reserved: at D = 128 this is 231,584 of the
+  // 232,448 bytes a CTA may use.
+  static constexpr int kSmemBytes = 2 * kTileBytes + kQStages * kTileBytes + kDoStages * kTileBytes + kDsBytes +
+                                    kDqStages * kDqChunkBytes + kQStages * kVecBytes + 8 * kNumBars + 16;
   static constexpr int kThreads = 512;
   static constexpr bool kAliasDq = (D == 128);
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static constexpr uint32_t kColDQ = kAliasDq ? 128 : 256 + 2 * D;
 };
+static_assert(BwdCfg<128>::kSmemBytes <= 232448, "backward shared memory over the per-CTA limit");
 
 // ---------------------------------------------------------------- preprocess
 // Half a warp per row (16 lanes x 16 bytes of O and of dO for D = 128, two rows
@@ -132,7 +144,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p)
     const bool in = row < rows;
     const size_t bh = in ? row / p.Np : 0;
     const int n = in ? static_cast<int>(row % p.Np) : 0;
-    if (in) {  // zero this row's slice of the dQ accumulator (row layout is irrelevant for zeros)
+    if (in) {  // zero D floats of the dQ accumulator (every float is zeroed once, whatever the layout)
       float4* acc = reinterpret_cast<float4*>(p.dqacc + row * D);
       acc[2 * part] = make_float4(0.f, 0.f, 0.f, 0.f);
       acc[2 * part + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -163,43 +175,43 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p)
     for (int off = kLanesPerRow / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (in && part == 0) {
       // tile padding or a padded token: D = 0 and LSE = +inf, so its P is exactly 0
-      p.Drow[row] = valid ? s : 0.f;
-      p.lse2[row] = valid ? p.lse[bh * p.N + n] * 1.4426950408889634f : INFINITY;
+      p.nD[row] = valid ? -s : 0.f;
+      p.nlse2[row] = valid ? -p.lse[bh * p.N + n] * 1.4426950408889634f : -INFINITY;
     }
   }
 }
 
 // ---------------------------------------------------------------- dQ accumulator layout
-// Rows are taken in groups of 32 (row n = 32 g + l).  Inside a group, the
-// 16-byte unit u (columns 4u..4u+3) of the 32 rows is stored contiguously, row
-// l at offset 16 l: element (n, c) of head bh sits at float index
-//   ((bh * Np/32 + g) * D/4 + c/4) * 128 + 4 l + c % 4.
-// A warp whose lane l owns row 32 g + l then adds unit u of all 32 rows with
-// one coalesced 512-byte vector reduction.
+// The partial dQ tile of one (query tile, key tile) pair is reduced as D / 32
+// chunks of 128 rows x 32 columns (16 KB, contiguous in the accumulator so that
+// one bulk reduce-add covers it).  Inside a chunk, row r holds its 32 floats in
+// eight 16-byte units, unit u stored at position u ^ (r % 8): the drain's
+// shared-memory writes (one row per thread) then spread over all banks.
+// Element (n, c) of head bh sits at float index
+//   dqacc_chunk(bh, ntiles, n / 128, c / 32) + (n % 128) * 32
+//     + (((c % 32) / 4) ^ (n % 8)) * 4 + c % 4.
 template <int D>
-__device__ __forceinline__ size_t dqacc_unit(size_t bh, int Np, int g, int u) {
-  return ((bh * static_cast<size_t>(Np / 32) + g) * (D / 4) + u) * 128;
+__device__ __forceinline__ size_t dqacc_chunk(size_t bh, int ntiles, int tile, int chunk) {
+  return ((bh * static_cast<size_t>(ntiles) + tile) * (D / 32) + chunk) * 4096;
 }
 
 // ---------------------------------------------------------------- dQ convert
-// One block per 32-row group: coalesced reads of the interleaved accumulator,
-// a transpose through shared memory, coalesced bf16 row writes of scale * acc.
+// One block per 32-row group: coalesced reads of the chunked accumulator, a
+// transpose through shared memory, coalesced bf16 row writes of scale * acc.
 template <int D, bool kStrided = false>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs<kStrided> p) {
   __shared__ float tile[32][D + 4];
   const int groups = p.Np / 32;
   const size_t bh = blockIdx.x / groups;
   const int g = static_cast<int>(blockIdx.x % groups);
-  const float4* src = reinterpret_cast<const float4*>(p.dqacc + dqacc_unit<D>(bh, p.Np, g, 0));
+  const int t128 = g >> 2, r0 = (g & 3) * 32;  // 128-row tile and first row inside it
 #pragma unroll
-  for (int k = 0; k < D / 32; ++k) {  // 32 * D / 4 float4 per group, 256 threads
-    const int f = threadIdx.x + 256 * k;
-    const int u = f >> 5, l = f & 31;
-    const float4 a = src[f];
-    tile[l][4 * u + 0] = a.x;
-    tile[l][4 * u + 1] = a.y;
-    tile[l][4 * u + 2] = a.z;
-    tile[l][4 * u + 3] = a.w;
+  for (int c = 0; c < D / 32; ++c) {  // 32 rows x 8 units of one chunk: 256 float4, one per thread
+    const int rr = threadIdx.x >> 3, up = threadIdx.x & 7;
+    const int u = up ^ (rr & 7);  // r0 is a multiple of 8, so (r0 + rr) % 8 = rr % 8
+    const float4 a = reinterpret_cast<const float4*>(p.dqacc + dqacc_chunk<D>(bh, p.ntiles, t128, c) +
+                                                     static_cast<size_t>(r0) * 32)[threadIdx.x];
+    *reinterpret_cast<float4*>(&tile[rr][c * 32 + 4 * u]) = a;
   }
   __syncthreads();
 #pragma unroll
@@ -221,12 +233,6 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs<kStrided> p) 
   }
 }
 
-__device__ __forceinline__ void red_add_v4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(a)),
-               "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
-               : "memory");
-}
-
 // Writes 32 fp32 values of row r (columns c..c+31 of a D-wide row), converted to
 // bf16, into a 128-row tile staged in the TMA 128-byte-swizzled layout.
 __device__ __forceinline__ void stage_row32_bf16(uint8_t* tile, int r, int c, const uint32_t (&v)[32], float mul) {
@@ -243,24 +249,25 @@ __device__ __forceinline__ void stage_row32_bf16(uint8_t* tile, int r, int c, co
 }
 
 // P^T = 2^(S^T * scale_log2 - LSE_q * log2 e) for one key row and 64 query
-// columns (LSE values broadcast from shared memory, 16 bytes per load).
+// columns, in place (x holds the raw scores on entry, the weights on exit).
+// The negated LSE values are broadcast from shared memory, 16 bytes per load.
 // kPoly: one pair in four on the FMA pipe (exp2_poly2), unmasked tiles only.
 template <bool kPoly>
-__device__ __forceinline__ void exp_cols64(const uint32_t (&sv)[64], const float* Lv, float sl2, float (&pv)[64]) {
+__device__ __forceinline__ void exp_cols64(float (&x)[64], const float* nLv, float sl2) {
+  const uint64_t sl2x2 = f2(sl2, sl2);
 #pragma unroll
   for (int c4 = 0; c4 < 16; ++c4) {
-    const float4 l4 = reinterpret_cast<const float4*>(Lv)[c4];
-    const float x0 = fmaf(__uint_as_float(sv[4 * c4 + 0]), sl2, -l4.x);
-    const float x1 = fmaf(__uint_as_float(sv[4 * c4 + 1]), sl2, -l4.y);
-    const float x2 = fmaf(__uint_as_float(sv[4 * c4 + 2]), sl2, -l4.z);
-    const float x3 = fmaf(__uint_as_float(sv[4 * c4 + 3]), sl2, -l4.w);
-    pv[4 * c4 + 0] = fast_exp2(x0);
-    pv[4 * c4 + 1] = fast_exp2(x1);
+    const float4 l4 = reinterpret_cast<const float4*>(nLv)[c4];
+    float a0, a1, a2, a3;
+    f2_split(ffma2(f2(x[4 * c4 + 0], x[4 * c4 + 1]), sl2x2, f2(l4.x, l4.y)), a0, a1);
+    f2_split(ffma2(f2(x[4 * c4 + 2], x[4 * c4 + 3]), sl2x2, f2(l4.z, l4.w)), a2, a3);
+    x[4 * c4 + 0] = fast_exp2(a0);
+    x[4 * c4 + 1] = fast_exp2(a1);
     if (kPoly && (c4 & 1)) {
-      exp2_poly2(x2, x3, pv[4 * c4 + 2], pv[4 * c4 + 3]);
+      exp2_poly2(a2, a3, x[4 * c4 + 2], x[4 * c4 + 3]);
     } else {
-      pv[4 * c4 + 2] = fast_exp2(x2);
-      pv[4 * c4 + 3] = fast_exp2(x3);
+      x[4 * c4 + 2] = fast_exp2(a2);
+      x[4 * c4 + 3] = fast_exp2(a3);
     }
   }
 }
@@ -280,14 +287,18 @@ __global__ void __launch_bounds__(512, 1)
   }
   uint8_t* sK = smem_raw;
   uint8_t* sV = smem_raw + C::kTileBytes;
-  uint8_t* sStage = smem_raw + 2 * C::kTileBytes;  // stage s: Q at +0, dO at +kTileBytes
-  uint8_t* sDS = sStage + C::kStages * 2 * C::kTileBytes;
-  uint8_t* sVec = sDS + C::kDsBytes;  // stage s: LSE*log2(e) [128] then D [128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sVec + C::kStages * C::kVecBytes);
+  uint8_t* sQ = smem_raw + 2 * C::kTileBytes;              // Q stage s at s * kTileBytes
+  uint8_t* sDO = sQ + C::kQStages * C::kTileBytes;        // dO stage s at s * kTileBytes
+  uint8_t* sDS = sDO + C::kDoStages * C::kTileBytes;
+  uint8_t* sDQ = sDS + C::kDsBytes;                        // dQ staging buffers, kDqChunkBytes each
+  uint8_t* sVec = sDQ + C::kDqStages * C::kDqChunkBytes;  // Q stage s: -LSE*log2(e) [128] then -D [128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sVec + C::kQStages * C::kVecBytes);
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
-  uint64_t* q_empty = bars + 1 + C::kStages;
-  uint64_t* s_full = bars + 1 + 2 * C::kStages;
+  uint64_t* q_empty = q_full + C::kQStages;
+  uint64_t* do_full = q_empty + C::kQStages;
+  uint64_t* do_empty = do_full + C::kDoStages;
+  uint64_t* s_full = do_empty + C::kDoStages;
   uint64_t* dp_full = s_full + 1;
   uint64_t* p_full = s_full + 2;
   uint64_t* ds_full = s_full + 3;
@@ -295,6 +306,8 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* dq_empty = s_full + 5;
   uint64_t* kv_done = s_full + 6;
   uint64_t* epi_bar = s_full + 7;
+  uint64_t* a_idle = s_full + 8;  // stream A: every product it issued has completed
+  uint64_t* b_idle = s_full + 9;  // stream B: the same
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -354,9 +367,13 @@ __global__ void __launch_bounds__(512, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
-    for (int i = 0; i < C::kStages; ++i) {
+    for (int i = 0; i < C::kQStages; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 2);  // one commit from each MMA stream
+    }
+    for (int i = 0; i < C::kDoStages; ++i) {
+      mbar_init(&do_full[i], 1);
+      mbar_init(&do_empty[i], 2);  // dP^T (stream B) and dV (stream A) have read it
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -366,6 +383,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(dq_empty, 128);
     mbar_init(kv_done, 2);  // dV (stream A) and dK (stream B) complete
     mbar_init(epi_bar, 128);
+    mbar_init(a_idle, 1);
+    mbar_init(b_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -377,67 +396,89 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) FA_TRACE_AT(6, 0, 0);
 
   if (warp >= 12) {
     regs_dec<64>();
     if (warp == 13 && lane == 0) {
-      // ---------------------------------------------------------- producer
+      // ---------------------------------------------------------- producer: K, V, then Q + LSE + D
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      prefetch_tmap(&tmdO);
-      mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
-      for (int c = 0; c < C::kChunks; ++c) {
-        if constexpr (kStrided) {
-          tma_load_tile(&tmK, p.map4 & kBMapK, kv_full, sK + c * 16384, c * 64, k0, bkv, kh, b);
-          tma_load_tile(&tmV, p.map4 & kBMapV, kv_full, sV + c * 16384, c * 64, k0, bkv, kh, b);
-        } else {
-          tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, k0, bkv);
-          tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, k0, bkv);
-        }
-      }
-      int issued[C::kStages];
-#pragma unroll
-      for (int i = 0; i < C::kStages; ++i) issued[i] = 0;
-      QCursor cur = first();
-      for (int it = 0; it < total; ++it, cur = advance(cur)) {
-        const int s = it % C::kStages;
-        if (!mbar_wait(&q_empty[s], ((it / C::kStages) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&q_full[s], 2 * C::kTileBytes + C::kVecBytes);
-        const int row0 = cur.i * 128, bh = bh0 + cur.hq;
-        uint8_t* st = sStage + s * 2 * C::kTileBytes;
+      const bool stall = g_debug_stall != 0;  // test hook: K/V never arrive
+      if (!stall) {
+        mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c) {
           if constexpr (kStrided) {
-            const int hq = kh * p.g + cur.hq;
-            tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, row0, bh, hq, b);
-            tma_load_tile(&tmdO, p.map4 & kBMapDO, &q_full[s], st + C::kTileBytes + c * 16384, c * 64, row0, bh, hq,
-                          b);
+            tma_load_tile(&tmK, p.map4 & kBMapK, kv_full, sK + c * 16384, c * 64, k0, bkv, kh, b);
+            tma_load_tile(&tmV, p.map4 & kBMapV, kv_full, sV + c * 16384, c * 64, k0, bkv, kh, b);
           } else {
-            tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
-            tma_load_3d(&tmdO, &q_full[s], st + C::kTileBytes + c * 16384, c * 64, row0, bh);
+            tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, k0, bkv);
+            tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, k0, bkv);
           }
         }
+      }
+      int issued[C::kQStages];
+#pragma unroll
+      for (int i = 0; i < C::kQStages; ++i) issued[i] = 0;
+      QCursor cur = first();
+      for (int it = 0; it < total; ++it, cur = advance(cur)) {
+        const int s = it % C::kQStages;
+        if (!mbar_wait(&q_empty[s], ((it / C::kQStages) & 1) ^ 1, abort_flag)) break;
+        FA_TRACE_AT(5, it, 0);
+        mbar_arrive_expect_tx(&q_full[s], C::kTileBytes + C::kVecBytes);
+        const int row0 = cur.i * 128, bh = bh0 + cur.hq;
+        uint8_t* st = sQ + s * C::kTileBytes;
+        for (int c = 0; c < C::kChunks; ++c) {
+          if constexpr (kStrided)
+            tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, row0, bh, kh * p.g + cur.hq,
+                          b);
+          else
+            tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
+        }
         const size_t vrow = static_cast<size_t>(bh) * p.Np + row0;
-        bulk_load(sVec + s * C::kVecBytes, p.lse2 + vrow, 512, &q_full[s]);
-        bulk_load(sVec + s * C::kVecBytes + 512, p.Drow + vrow, 512, &q_full[s]);
+        bulk_load(sVec + s * C::kVecBytes, p.nlse2 + vrow, 512, &q_full[s]);
+        bulk_load(sVec + s * C::kVecBytes + 512, p.nD + vrow, 512, &q_full[s]);
         ++issued[s];
       }
-      const unsigned long long t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(kv_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      // Never leave the CTA with copies still landing in shared memory.
+      if (!stall) mbar_wait_drain(kv_full, 0);
+      for (int s = 0; s < C::kQStages; ++s)
+        if (issued[s] > 0) mbar_wait_drain(&q_full[s], (issued[s] - 1) & 1);
+    } else if (warp == 15 && lane == 0) {
+      // ---------------------------------------------------------- producer: dO
+      prefetch_tmap(&tmdO);
+      int issued[C::kDoStages];
+#pragma unroll
+      for (int i = 0; i < C::kDoStages; ++i) issued[i] = 0;
+      QCursor cur = first();
+      for (int it = 0; it < total; ++it, cur = advance(cur)) {
+        const int s = it % C::kDoStages;
+        if (!mbar_wait(&do_empty[s], ((it / C::kDoStages) & 1) ^ 1, abort_flag)) break;
+        FA_TRACE_AT(5, it, 1);
+        mbar_arrive_expect_tx(&do_full[s], C::kTileBytes);
+        const int row0 = cur.i * 128, bh = bh0 + cur.hq;
+        uint8_t* st = sDO + s * C::kTileBytes;
+        for (int c = 0; c < C::kChunks; ++c) {
+          if constexpr (kStrided)
+            tma_load_tile(&tmdO, p.map4 & kBMapDO, &do_full[s], st + c * 16384, c * 64, row0, bh,
+                          kh * p.g + cur.hq, b);
+          else
+            tma_load_3d(&tmdO, &do_full[s], st + c * 16384, c * 64, row0, bh);
+        }
+        ++issued[s];
       }
-      for (int s = 0; s < C::kStages; ++s)
-        if (issued[s] > 0)
-          while (!mbar_try_wait(smem_u32(&q_full[s]), (issued[s] - 1) & 1) &&
-                 globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
+      for (int s = 0; s < C::kDoStages; ++s)
+        if (issued[s] > 0) mbar_wait_drain(&do_full[s], (issued[s] - 1) & 1);
     } else if ((warp == 12 || warp == 14) && lane == 0) {
       // ---------------------------------------------------------- MMA issuers
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aSt = smem_u32(sStage), aDS = smem_u32(sDS);
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
+                     aDS = smem_u32(sDS);
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, false, true);     // dV, dK (A from TMEM)
       constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);      // dQ = dS K
-      auto st_q = [&](int s) { return aSt + s * 2 * C::kTileBytes; };
-      auto st_do = [&](int s) { return aSt + s * 2 * C::kTileBytes + C::kTileBytes; };
+      auto st_q = [&](int s) { return aQ + s * C::kTileBytes; };
+      auto st_do = [&](int s) { return aDO + s * C::kTileBytes; };
       // X^T = A B^T with both operands K-major: A = K or V (rows = keys), B = Q or dO.
       auto kmajor_nt = [&](uint32_t dcol, uint32_t a, uint32_t bb) {
 #pragma unroll
@@ -453,40 +494,50 @@ __global__ void __launch_bounds__(512, 1)
           umma_ts(tmem + dcol, tmem + acol + (k >> 2) * 64 + (k & 3) * 8,
                   sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
       };
-      bool ok = mbar_wait(kv_full, 0, abort_flag) && (total == 0 || mbar_wait(&q_full[0], 0, abort_flag));
+      bool ok = mbar_wait(kv_full, 0, abort_flag);
       if (warp == 12) {
         // stream A: S^T_i = K Q_i^T, then dV += P_i^T dO_i once P_i is in TMEM
-        if (ok && total > 0) {
+        if (ok && total > 0 && (ok = mbar_wait(&q_full[0], 0, abort_flag))) {
           tc_fence_after();
           kmajor_nt(C::kColS, aK, st_q(0));
           umma_commit(s_full);
         }
         for (int it = 0; ok && it < total; ++it) {
-          const int s = it % C::kStages;
-          const int s1 = (it + 1) % C::kStages;
+          const int s = it % C::kQStages, s1 = (it + 1) % C::kQStages, so = it % C::kDoStages;
           if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
+          FA_TRACE_AT(2, it, 0);
+          if (!(ok = mbar_wait(&do_full[so], (it / C::kDoStages) & 1, abort_flag))) break;
           tc_fence_after();
-          ts_acc(C::kColDV, C::kColS, st_do(s), it > 0);  // dV += P^T dO
-          umma_commit(&q_empty[s]);
+          ts_acc(C::kColDV, C::kColS, st_do(so), it > 0);  // dV += P^T dO
+          umma_commit(&do_empty[so]);
+          umma_commit(&q_empty[s]);  // S^T of this tile (issued earlier) has read Q
+          FA_TRACE_AT(2, it, 1);
           if (it + 1 < total) {
-            if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kQStages) & 1, abort_flag))) break;
+            FA_TRACE_AT(2, it, 2);
             tc_fence_after();
             kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
             umma_commit(s_full);
+            FA_TRACE_AT(2, it, 3);
           }
         }
         if (ok) umma_commit(kv_done);
+        // Before the CTA frees TMEM: every product this thread issued has completed.
+        umma_commit(a_idle);
+        mbar_wait_drain(a_idle, 0);
       } else {
         // stream B: dP^T_i = V dO_i^T; once dS_i is ready dK += dS_i^T Q_i and dQ_i = dS_i K
-        if (ok && total > 0) {
+        if (ok && total > 0 && (ok = mbar_wait(&do_full[0], 0, abort_flag))) {
           tc_fence_after();
           kmajor_nt(C::kColDP, aV, st_do(0));
           umma_commit(dp_full);
+          umma_commit(&do_empty[0]);
         }
         for (int it = 0; ok && it < total; ++it) {
-          const int s = it % C::kStages;
-          const int s1 = (it + 1) % C::kStages;
+          const int s = it % C::kQStages, so1 = (it + 1) % C::kDoStages;
           if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
+          FA_TRACE_AT(3, it, 0);
+          if (!(ok = mbar_wait(&q_full[s], (it / C::kQStages) & 1, abort_flag))) break;
           tc_fence_after();
           ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
           if (!C::kAliasDq && it > 0) {
@@ -499,17 +550,23 @@ __global__ void __launch_bounds__(512, 1)
                     sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
           umma_commit(dq_full);
           umma_commit(&q_empty[s]);
+          FA_TRACE_AT(3, it, 1);
           if (it + 1 < total) {
             if (C::kAliasDq) {
               if (!(ok = mbar_wait(dq_empty, it & 1, abort_flag))) break;
             }
-            if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait(&do_full[so1], ((it + 1) / C::kDoStages) & 1, abort_flag))) break;
+            FA_TRACE_AT(3, it, 2);
             tc_fence_after();
-            kmajor_nt(C::kColDP, aV, st_do(s1));  // dP^T of the next query tile
+            kmajor_nt(C::kColDP, aV, st_do(so1));  // dP^T of the next query tile
             umma_commit(dp_full);
+            umma_commit(&do_empty[so1]);
+            FA_TRACE_AT(3, it, 3);
           }
         }
         if (ok) umma_commit(kv_done);
+        umma_commit(b_idle);
+        mbar_wait_drain(b_idle, 0);
       }
     }
     __syncwarp();
@@ -530,25 +587,32 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     QCursor cur = first();
     for (int it = 0; it < total; ++it, cur = advance(cur)) {
-      const int s = it % C::kStages;
+      const int s = it % C::kQStages;
       const int q0 = cur.i * 128 + 64 * w;  // first query of my columns
-      const float* Lv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes) + 64 * w;
-      const float* Dv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes + 512) + 64 * w;
+      const float* nLv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes) + 64 * w;
+      const float* nDv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes + 512) + 64 * w;
       bool full = tile_valid;  // every (query, key) pair of my 64 columns allowed?
       if (p.causal) full = full && (k0 + 127 <= q0);
       if (p.window >= 0) full = full && (q0 + 63 - k0 <= p.window) && (k0 + 127 - q0 <= p.window);
-      if (!(ok = mbar_wait(&q_full[s], (it / C::kStages) & 1, abort_flag))) break;  // LSE / D landed
-      if (!(ok = mbar_wait(s_full, it & 1, abort_flag))) break;
+      // (warp-uniform outcomes: the TMEM loads and stores below are warp-collective)
+      ok = mbar_wait(&q_full[s], (it / C::kQStages) & 1, abort_flag);  // LSE / D landed
+      ok = ok && mbar_wait(s_full, it & 1, abort_flag);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 0);
       tc_fence_after();
-      uint32_t sv[64];
-      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_wait_ld();
-      float pv[64];
+      float pv[64];  // the fp32 weights P^T of my 64 columns
+      {
+        uint32_t sv[64];
+        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 64; ++c) pv[c] = __uint_as_float(sv[c]);
+      }
       if (full)
-        exp_cols64<true>(sv, Lv, sl2, pv);
+        exp_cols64<true>(pv, nLv, sl2);
       else
-        exp_cols64<false>(sv, Lv, sl2, pv);
+        exp_cols64<false>(pv, nLv, sl2);
       if (!full) {  // tiles on the diagonal / window edge only: one branch, not one per element
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -559,15 +623,20 @@ __global__ void __launch_bounds__(512, 1)
           pv[c] = keep ? pv[c] : 0.f;
         }
       }
-      uint32_t pk[32];  // my 64 P^T values, packed bf16
+      {
+        uint32_t pk[32];  // my 64 P^T values, packed bf16: the A operand of dV += P^T dO
 #pragma unroll
-      for (int u = 0; u < 32; ++u) pk[u] = pack_bf16x2(pv[2 * u], pv[2 * u + 1]);
-      tmem_st32(tS, pk);
+        for (int u = 0; u < 32; ++u) pk[u] = pack_bf16x2(pv[2 * u], pv[2 * u + 1]);
+        tmem_st32(tS, pk);
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
+      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 1);
 
-      if (!(ok = mbar_wait(dp_full, it & 1, abort_flag))) break;
+      ok = mbar_wait(dp_full, it & 1, abort_flag);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 2);
       tc_fence_after();
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -577,16 +646,18 @@ __global__ void __launch_bounds__(512, 1)
         uint32_t ds[16];
 #pragma unroll
         for (int u2 = 0; u2 < 8; ++u2) {
-          const float4 d4 = reinterpret_cast<const float4*>(Dv)[8 * h + u2];
-          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int u = 2 * u2 + e;
-            const uint32_t pp = pk[h * 16 + u];
-            const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xffff0000u);
-            ds[u] = pack_bf16x2(p0 * (__uint_as_float(dv[2 * u]) - dd[2 * e]),
-                                p1 * (__uint_as_float(dv[2 * u + 1]) - dd[2 * e + 1]));
-          }
+          const float4 d4 = reinterpret_cast<const float4*>(nDv)[8 * h + u2];
+          // dS = P (dP - D) on packed pairs, P kept in fp32 since the exponent phase
+          const int c = 32 * h + 4 * u2;
+          float a0, a1, a2, a3;
+          f2_split(fmul2(f2(pv[c], pv[c + 1]),
+                         fadd2(f2(__uint_as_float(dv[4 * u2]), __uint_as_float(dv[4 * u2 + 1])), f2(d4.x, d4.y))),
+                   a0, a1);
+          f2_split(fmul2(f2(pv[c + 2], pv[c + 3]),
+                         fadd2(f2(__uint_as_float(dv[4 * u2 + 2]), __uint_as_float(dv[4 * u2 + 3])), f2(d4.z, d4.w))),
+                   a2, a3);
+          ds[2 * u2] = pack_bf16x2(a0, a1);
+          ds[2 * u2 + 1] = pack_bf16x2(a2, a3);
         }
         // dS^T (packed) over dP^T columns this thread has already read; dS into
         // shared memory as rows = keys, columns = queries (MN-major A of dQ).
@@ -602,39 +673,55 @@ __global__ void __launch_bounds__(512, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(ds_full);
+      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 3);
     }
   } else {
     // ------------------------------------------------------------ dQ drain, then dK/dV epilogue
     regs_inc<160>();
     const int wl = warp & 3;
-    const int r = wl * 32 + lane;
+    const int r = wl * 32 + lane;  // query row of the dQ tile (drain), key row (epilogue)
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
+    constexpr int kBarDrain = 1, kBarDrainAnd = 2;  // named barriers of the 128 drain threads
     bool ok = true;
+    int nchunk = 0;  // chunks handed to the TMA unit so far
     QCursor cur = first();
     for (int it = 0; it < total; ++it, cur = advance(cur)) {
-      if (!(ok = mbar_wait(dq_full, it & 1, abort_flag))) break;
+      ok = mbar_wait(dq_full, it & 1, abort_flag);
+      // all 128 threads take the same branch: the named barriers below need every one of them
+      if (!(ok = named_bar_and(kBarDrainAnd, 128, ok))) break;
+      if (r == 0) FA_TRACE_AT(4, it, 0);
       tc_fence_after();
-      // my row is 32 * (4 * i + wl) + lane: group 4 * i + wl, slot `lane`
-      float* dst = p.dqacc + dqacc_unit<D>(bh0 + cur.hq, p.Np, 4 * cur.i + wl, 0) + 4 * lane;
       uint32_t v[D];
 #pragma unroll
       for (int c = 0; c < D / 32; ++c)
         tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(dq_empty);  // TMEM tile free before the reductions are issued
-      if (C::kAliasDq && it + 1 < total) {
-        // Hold the row until the next dS has been written: the reductions then
-        // overlap the exponent phase instead of competing with the dS stores to
-        // shared memory.  Phase (it + 1) of ds_full cannot be overtaken: the
-        // phase after it needs dP^T of it + 2, which waits for this tile's
-        // dq_empty (the dQ tile aliases the dP^T columns when D = 128).
-        if (!(ok = mbar_wait(ds_full, (it + 1) & 1, abort_flag))) break;
-      }
+      mbar_arrive(dq_empty);  // TMEM tile free before the reductions are staged
+      if (r == 0) FA_TRACE_AT(4, it, 1);
+      const size_t bh = static_cast<size_t>(bh0 + cur.hq);
 #pragma unroll
-      for (int c = 0; c < D; c += 4) red_add_v4(dst + 32 * c, v[c], v[c + 1], v[c + 2], v[c + 3]);
+      for (int c = 0; c < C::kDqChunks; ++c, ++nchunk) {
+        uint8_t* buf = sDQ + (nchunk % C::kDqStages) * C::kDqChunkBytes;
+        // the buffer's previous chunk has been read by the TMA unit
+        if (r == 0 && nchunk >= C::kDqStages) bulk_wait_read<C::kDqStages - 1>();
+        named_bar_sync(kBarDrain, 128);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          *reinterpret_cast<uint4*>(buf + r * 128 + ((u ^ (r & 7)) << 4)) =
+              make_uint4(v[c * 32 + 4 * u], v[c * 32 + 4 * u + 1], v[c * 32 + 4 * u + 2], v[c * 32 + 4 * u + 3]);
+        fence_proxy_async_smem();
+        named_bar_sync(kBarDrain, 128);
+        if (r == 0) {
+          bulk_reduce_add_f32(p.dqacc + dqacc_chunk<D>(bh, p.ntiles, cur.i, c), buf, C::kDqChunkBytes);
+          bulk_commit();
+        }
+      }
+      if (r == 0) FA_TRACE_AT(4, it, 2);
     }
+    if (r == 0) bulk_wait0();  // every reduction complete before the CTA exits
     if (ok) ok = mbar_wait(kv_done, 0, abort_flag);
+    ok = named_bar_and(kBarDrainAnd, 128, ok);  // the TMEM loads below are warp-collective
     if (ok) {
       tc_fence_after();
       // K and V tiles are no longer read: stage dV over V and dK over K.
@@ -674,6 +761,7 @@ __global__ void __launch_bounds__(512, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) FA_TRACE_AT(6, 0, 1);
   if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -149,7 +149,17 @@ bool set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
 }
 
-inline fa_status launched() { return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+// Launches one kernel and reports that launch's own outcome (an error left
+// behind by an earlier, unrelated call is not taken for this one).
+template <typename... KArgs, typename... Args>
+fa_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 fa::SimtParams simt_params(int B, int H, int Hkv, int N, float scale, int causal, int window) {
   fa::SimtParams s{};
@@ -185,6 +195,7 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
                    float scale, int causal, int window, cudaStream_t st, const Layouts* L = nullptr, int splits = 0,
                    void* ws = nullptr, const uint8_t* bmask = nullptr, long long bmask_hs = 0,
                    const int* seqlens = nullptr) {
+  fa_status ls = FA_OK;
   using C = fa::FwdCfg<D>;
   const Layouts lay = L ? *L : contiguous_layouts(B, H, Hkv, N, D);
   CUtensorMap tq, tk, tv, to;
@@ -227,18 +238,18 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
     ps.map4 = (f4[0] ? fa::kMapQ : 0u) | (f4[1] ? fa::kMapK : 0u) | (f4[2] ? fa::kMapV : 0u) |
               (f4[3] ? fa::kMapO : 0u);
     mark_start(st);
-    fa::fwd_sm100_kernel<D, false, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, ps);
+    ls = launch(fa::fwd_sm100_kernel<D, false, false, true>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv, to, ps);
     mark_stop(st);
-    return launched();
+    return ls;
   }
   if (splits == 0) {
     mark_start(st);
     if (bmask)
-      fa::fwd_sm100_kernel<D, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+      ls = launch(fa::fwd_sm100_kernel<D, false, true>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv, to, p);
     else
-      fa::fwd_sm100_kernel<D, false, false><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+      ls = launch(fa::fwd_sm100_kernel<D, false, false>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv, to, p);
     mark_stop(st);
-    return launched();
+    return ls;
   }
   p.splits = splits;
   p.nq2 = p.npairs * 256;
@@ -246,12 +257,12 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
   p.part_m = reinterpret_cast<float4*>(static_cast<uint8_t*>(ws) +
                                        align256(static_cast<size_t>(splits) * B * H * p.nq2 * D * 4));
   mark_start(st);
-  fa::fwd_sm100_kernel<D, true, false><<<grid * splits, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+  ls = launch(fa::fwd_sm100_kernel<D, true, false>, grid * splits, C::kThreads, C::kSmemBytes, st, tq, tk, tv, to, p);
   mark_stop(st);
-  if (launched() != FA_OK) return FA_ERR_CUDA;
+  if (ls != FA_OK) return ls;
   const unsigned cgrid = static_cast<unsigned>(B * H) * ((N + 31) / 32);
-  fa::fwd_combine_kernel<D><<<cgrid, 256, 0, st>>>(p, o);
-  return launched();
+  ls = launch(fa::fwd_combine_kernel<D>, cgrid, 256, 0, st, p, o);
+  return ls;
 }
 
 // Fewer queries than keys (decode): Nq query rows at positions Nk - Nq + i
@@ -263,6 +274,7 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
 template <int D>
 fa_status fwd_decode_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
                           int Nq, int Nk, float scale, int causal, int window, cudaStream_t st, int splits, void* ws) {
+  fa_status ls = FA_OK;
   using C = fa::FwdCfg<D>;
   const int g = H / Hkv, Nv = g * Nq;  // rows of a virtual head
   CUtensorMap tq, tk, tv, to;
@@ -300,12 +312,13 @@ fa_status fwd_decode_bf16(const void* q, const void* k, const void* v, void* o, 
                                        align256(static_cast<size_t>(splits) * B * Hkv * p.nq2 * D * 4));
   const unsigned grid = static_cast<unsigned>(p.npairs) * B * Hkv * splits;
   mark_start(st);
-  fa::fwd_sm100_kernel<D, true, false, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, p);
+  ls = launch(fa::fwd_sm100_kernel<D, true, false, false, true>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv,
+              to, p);
   mark_stop(st);
-  if (launched() != FA_OK) return FA_ERR_CUDA;
+  if (ls != FA_OK) return ls;
   const unsigned cgrid = static_cast<unsigned>(B * Hkv) * ((Nv + 31) / 32);
-  fa::fwd_combine_kernel<D><<<cgrid, 256, 0, st>>>(static_cast<const fa::FwdParams&>(p), o);
-  return launched();
+  ls = launch(fa::fwd_combine_kernel<D>, cgrid, 256, 0, st, static_cast<const fa::FwdParams&>(p), o);
+  return ls;
 }
 
 void set_simt_strides(fa::SimtParams& s, const Layouts& L) {
@@ -323,6 +336,7 @@ template <int D>
 fa_status fwd_f32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                   float scale, int causal, int window, cudaStream_t st, const Layouts* L = nullptr,
                   const uint8_t* bmask = nullptr, long long bmask_hs = 0, const int* seqlens = nullptr) {
+  fa_status ls = FA_OK;
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
   set_simt_strides(s, L ? *L : contiguous_layouts(B, H, Hkv, N, D));
   s.bmask = bmask;
@@ -336,25 +350,25 @@ fa_status fwd_f32(const void* q, const void* k, const void* v, void* o, float* l
   s.lse_out = lse;
   dim3 grid((N + fa::kSimtRows - 1) / fa::kSimtRows, B * H);
   mark_start(st);
-  fa::fwd_simt_f32_kernel<D><<<grid, 32 * fa::kSimtRows, 0, st>>>(s);
+  ls = launch(fa::fwd_simt_f32_kernel<D>, grid, 32 * fa::kSimtRows, 0, st, s);
   mark_stop(st);
-  return launched();
+  return ls;
 }
 
 struct WsLayout {
-  size_t lse2, drow, dqacc, total;
+  size_t nlse2, nd, dqacc, total;
 };
 WsLayout ws_layout(int B, int H, int N, int d, fa_dtype dtype) {
   WsLayout w{};
   if (dtype == FA_FP32) {
-    w.drow = 0;
+    w.nd = 0;
     w.total = align256(static_cast<size_t>(B) * H * N * 4);
     return w;
   }
   const size_t rows = static_cast<size_t>(B) * H * padded_rows(N);
-  w.lse2 = 0;
-  w.drow = align256(rows * 4);
-  w.dqacc = w.drow + align256(rows * 4);
+  w.nlse2 = 0;
+  w.nd = align256(rows * 4);
+  w.dqacc = w.nd + align256(rows * 4);
   w.total = w.dqacc + align256(rows * d * 4);
   return w;
 }
@@ -364,6 +378,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
                    void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
                    int window, cudaStream_t st, const Layouts* L = nullptr, const uint8_t* bmask = nullptr,
                    long long bmask_hs = 0, const int* seqlens = nullptr) {
+  fa_status ls = FA_OK;
   using C = fa::BwdCfg<D>;
   const WsLayout w = ws_layout(B, H, N, D, FA_BF16);
   const Layouts lay = L ? *L : contiguous_layouts(B, H, Hkv, N, D);
@@ -372,8 +387,8 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   p.lse = lse;
   p.o = o;
   p.dout = dout;
-  p.lse2 = reinterpret_cast<float*>(wb + w.lse2);
-  p.Drow = reinterpret_cast<float*>(wb + w.drow);
+  p.nlse2 = reinterpret_cast<float*>(wb + w.nlse2);
+  p.nD = reinterpret_cast<float*>(wb + w.nd);
   p.dqacc = reinterpret_cast<float*>(wb + w.dqacc);
   p.dq = dq;
   p.B = B;
@@ -421,26 +436,27 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
     ps.sdq = lay.dq;
     ps.map4 = (f4[0] ? fa::kBMapQ : 0u) | (f4[1] ? fa::kBMapK : 0u) | (f4[2] ? fa::kBMapV : 0u) |
               (f4[3] ? fa::kBMapDO : 0u) | (f4[4] ? fa::kBMapDK : 0u) | (f4[5] ? fa::kBMapDV : 0u);
-    fa::bwd_pre_kernel<D, true><<<pre_grid, 256, 0, st>>>(ps);
-    if (launched() != FA_OK) return FA_ERR_CUDA;
+    ls = launch(fa::bwd_pre_kernel<D, true>, pre_grid, 256, 0, st, ps);
+    if (ls != FA_OK) return ls;
     mark_start(st);
-    fa::bwd_sm100_kernel<D, false, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, ps);
+    ls = launch(fa::bwd_sm100_kernel<D, false, true>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv, tdo, tdk,
+                tdv, ps);
     mark_stop(st);
-    if (launched() != FA_OK) return FA_ERR_CUDA;
-    fa::bwd_dq_kernel<D, true><<<dq_grid, 256, 0, st>>>(ps);
-    return launched();
+    if (ls != FA_OK) return ls;
+    ls = launch(fa::bwd_dq_kernel<D, true>, dq_grid, 256, 0, st, ps);
+    return ls;
   }
-  fa::bwd_pre_kernel<D><<<pre_grid, 256, 0, st>>>(p);
-  if (launched() != FA_OK) return FA_ERR_CUDA;
+  ls = launch(fa::bwd_pre_kernel<D>, pre_grid, 256, 0, st, p);
+  if (ls != FA_OK) return ls;
   mark_start(st);
   if (bmask)
-    fa::bwd_sm100_kernel<D, true><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
+    ls = launch(fa::bwd_sm100_kernel<D, true>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv, tdo, tdk, tdv, p);
   else
-    fa::bwd_sm100_kernel<D, false><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, tdo, tdk, tdv, p);
+    ls = launch(fa::bwd_sm100_kernel<D, false>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv, tdo, tdk, tdv, p);
   mark_stop(st);
-  if (launched() != FA_OK) return FA_ERR_CUDA;
-  fa::bwd_dq_kernel<D><<<dq_grid, 256, 0, st>>>(p);
-  return launched();
+  if (ls != FA_OK) return ls;
+  ls = launch(fa::bwd_dq_kernel<D>, dq_grid, 256, 0, st, p);
+  return ls;
 }
 
 template <int D>
@@ -448,6 +464,7 @@ fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, co
                   void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
                   int window, cudaStream_t st, const Layouts* L = nullptr, const uint8_t* bmask = nullptr,
                   long long bmask_hs = 0, const int* seqlens = nullptr) {
+  fa_status ls = FA_OK;
   fa::SimtParams s = simt_params(B, H, Hkv, N, scale, causal, window);
   set_simt_strides(s, L ? *L : contiguous_layouts(B, H, Hkv, N, D));
   s.bmask = bmask;
@@ -465,17 +482,17 @@ fa_status bwd_f32(const void* q, const void* k, const void* v, const void* o, co
   s.dv = static_cast<float*>(dv);
   s.Drow = static_cast<float*>(ws);
   const size_t rows = static_cast<size_t>(B) * H * N;
-  fa::bwd_rowdot_f32_kernel<D><<<static_cast<unsigned>((rows + fa::kSimtRows - 1) / fa::kSimtRows),
-                                 32 * fa::kSimtRows, 0, st>>>(s);
-  if (launched() != FA_OK) return FA_ERR_CUDA;
+  ls = launch(fa::bwd_rowdot_f32_kernel<D>, static_cast<unsigned>((rows + fa::kSimtRows - 1) / fa::kSimtRows),
+              32 * fa::kSimtRows, 0, st, s);
+  if (ls != FA_OK) return ls;
   dim3 gkv((N + fa::kSimtRows - 1) / fa::kSimtRows, B * Hkv);
   mark_start(st);
-  fa::bwd_dkdv_f32_kernel<D><<<gkv, 32 * fa::kSimtRows, 0, st>>>(s);
+  ls = launch(fa::bwd_dkdv_f32_kernel<D>, gkv, 32 * fa::kSimtRows, 0, st, s);
   mark_stop(st);
-  if (launched() != FA_OK) return FA_ERR_CUDA;
+  if (ls != FA_OK) return ls;
   dim3 gq((N + fa::kSimtRows - 1) / fa::kSimtRows, B * H);
-  fa::bwd_dq_f32_kernel<D><<<gq, 32 * fa::kSimtRows, 0, st>>>(s);
-  return launched();
+  ls = launch(fa::bwd_dq_f32_kernel<D>, gq, 32 * fa::kSimtRows, 0, st, s);
+  return ls;
 }
 
 // ---------------------------------------------------------------- packed variable lengths
@@ -508,12 +525,26 @@ fa_status packed_layouts(int H, int Hkv, int len, int d, int es, Layouts* L) {
   return FA_OK;
 }
 
+// The kernels run on the current device, where the tensor maps are built and
+// the allocation-free scratch address is looked up: a stream of another device
+// is an argument error (the legacy default stream, NULL, is the current
+// device's).
+fa_status check_stream(void* stream) {
+  int cur = 0, sdev = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return FA_ERR_CUDA;
+  if (stream == nullptr) return FA_OK;
+  if (cudaStreamGetDevice(static_cast<cudaStream_t>(stream), &sdev) != cudaSuccess) return FA_ERR_INVALID_ARG;
+  return sdev == cur ? FA_OK : FA_ERR_INVALID_ARG;
+}
+
 // dtype / head-dimension dispatch shared by every entry point (arguments
 // already checked).
 fa_status run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                   int d, float scale, int causal, int window, fa_dtype dtype, void* stream, const Layouts* L,
                   int splits = 0, void* ws = nullptr, const uint8_t* bmask = nullptr, long long hs = 0,
                   const int* seqlens = nullptr) {
+  const fa_status sc = check_stream(stream);
+  if (sc != FA_OK) return sc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == FA_BF16)
     return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, N, scale, causal, window, st, L, splits, ws, bmask, hs,
@@ -529,6 +560,8 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* o, co
                   void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, int d, float scale, int causal,
                   int window, fa_dtype dtype, void* stream, const Layouts* L, const uint8_t* bmask = nullptr,
                   long long hs = 0, const int* seqlens = nullptr) {
+  const fa_status sc = check_stream(stream);
+  if (sc != FA_OK) return sc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == FA_BF16)
     return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, ws, B, H, Hkv, N, scale, causal, window, st, L,
@@ -723,6 +756,7 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
   if (!workspace || ws_bytes < decode_ws_bytes(B, H, Hkv, Nq, d, num_splits)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  if ((s = check_stream(stream)) != FA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return d == 64 ? fwd_decode_bf16<64>(q, k, v, o, lse, B, H, Hkv, Nq, Nk, scale, causal, window, st, num_splits,
                                        workspace)
@@ -811,6 +845,16 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  nullptr);
 }
 
+fa_status fa_debug_set_wait_limit(unsigned long long ns) {
+  const unsigned long long v = ns ? ns : fa::kWaitLimitNs;
+  return cudaMemcpyToSymbol(fa::g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_debug_set_stall(int on) {
+  const int v = on ? 1 : 0;
+  return cudaMemcpyToSymbol(fa::g_debug_stall, &v, sizeof(v)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status fa_last_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   unsigned int v = 0, zero = 0;
@@ -819,6 +863,20 @@ fa_status fa_last_device_status(void* stream) {
   if (v & fa::kStatusTimeout) return FA_ERR_TIMEOUT;
   return v ? FA_ERR_CUDA : FA_OK;
 }
+
+#ifdef FA_TRACE
+// Phase-timestamp builds only (not part of the ABI): copies or clears the trace buffer.
+constexpr size_t kTraceBytes =
+    sizeof(long long) * fa::kTraceCtas * fa::kTraceRoles * fa::kTraceIters * fa::kTraceEvents;
+int fa_trace_read(void* dst, size_t bytes) {
+  if (bytes > kTraceBytes) bytes = kTraceBytes;
+  return cudaMemcpyFromSymbol(dst, fa::g_trace, bytes) == cudaSuccess ? 0 : 1;
+}
+int fa_trace_clear(void) {
+  static long long zero[kTraceBytes / sizeof(long long)];
+  return cudaMemcpyToSymbol(fa::g_trace, zero, sizeof(zero)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 }  // extern "C"
 
@@ -857,6 +915,7 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
   fa_status s = check_common(B, H, Hkv, N, d, scale, window, dtype);
   if (s != FA_OK) return s;
   if (ws_layout(B, H, N, d, dtype).total > FA_BWD_NOALLOC_SCRATCH_BYTES) return FA_ERR_WORKSPACE;
+  if ((s = check_stream(stream)) != FA_OK) return s;  // the scratch address is the current device's
   void* scratch = nullptr;
   s = noalloc_scratch(&scratch);
   if (s != FA_OK) return s;

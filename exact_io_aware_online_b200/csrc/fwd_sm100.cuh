@@ -106,7 +106,7 @@ struct FwdCfg {
   static constexpr int kStages = (D == 128) ? 4 : 8;
   static constexpr int kSmemQ = 2 * kTileBytes;
   static constexpr int kSmemKV = kStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 8;
+  static constexpr int kNumBars = 1 + 2 * kStages + 9;
   static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + 8 * kNumBars + 16;
   static constexpr int kThreads = 384;
   static constexpr uint32_t kTmemCols = 512;
@@ -174,6 +174,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_full = s_full + 4;
   uint64_t* epi_bar = s_full + 6;  // softmax threads -> storing thread: O tile staged
+  uint64_t* mma_idle = s_full + 8;  // every product the MMA thread issued has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -250,6 +251,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&o_full[t], 1);
       mbar_init(&epi_bar[t], 128);
     }
+    mbar_init(mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -269,7 +271,8 @@ __global__ void __launch_bounds__(384, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      if (nkv > 0) {
+      const bool stall = g_debug_stall != 0;  // test hook: Q never arrives
+      if (nkv > 0 && !stall) {
         mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::kChunks; ++c)
@@ -302,14 +305,9 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       // Never leave the CTA with copies still landing in shared memory.
-      const unsigned long long t0 = globaltimer_ns();
-      while (nkv > 0 && !mbar_try_wait(smem_u32(q_full), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
-      }
+      if (nkv > 0 && !stall) mbar_wait_drain(q_full, 0);
       for (int s = 0; s < C::kStages; ++s)
-        if (issued[s] > 0)
-          while (!mbar_try_wait(smem_u32(&kv_full[s]), (issued[s] - 1) & 1) &&
-                 globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
+        if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
     } else if (warp == 8 && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       const uint32_t aQ = smem_u32(sQ), aKV = smem_u32(sKV);
@@ -372,6 +370,9 @@ __global__ void __launch_bounds__(384, 1)
           umma_commit(&o_full[t]);
         }
       }
+      // Before the CTA frees TMEM: every product this thread issued has completed.
+      umma_commit(mma_idle);
+      mbar_wait_drain(mma_idle, 0);
     }
     __syncwarp();
   } else {
@@ -402,7 +403,9 @@ __global__ void __launch_bounds__(384, 1)
       const int kv0 = jcur * 128;
       // block switched off for this query tile: every score of the tile is masked
       const bool block_off = kMask && !block_on(t, jcur);
-      if (!(ok = mbar_wait(&s_full[t], jj & 1, abort_flag))) break;
+      // (warp-uniform outcome: the TMEM loads and stores below are warp-collective)
+      ok = mbar_wait(&s_full[t], jj & 1, abort_flag);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
       tc_fence_after();
       if (kMask && block_off) {  // every weight of the tile is zero: store P = 0 and move on
         uint32_t z[16];
@@ -483,7 +486,7 @@ __global__ void __launch_bounds__(384, 1)
       const size_t sbh = static_cast<size_t>(split) * BH + bh;
       if (nkv_t <= 0) {
         p.part_m[sbh * p.nq2 + n] = make_float4(-INFINITY, 0.f, 0.f, 0.f);
-      } else if (ok && (ok = mbar_wait(&o_full[t], 0, abort_flag))) {
+      } else if (ok && (ok = __all_sync(0xffffffffu, mbar_wait(&o_full[t], 0, abort_flag)))) {
         tc_fence_after();
         float* dst = p.part_o + fwd_part_unit<D>(sbh, p.nq2, n >> 5, 0) + 4 * lane;
 #pragma unroll 1
@@ -502,6 +505,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else {
     if (ok && nkv > 0) ok = mbar_wait(&o_full[t], 0, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       const bool pad_row = qrow >= Lb;

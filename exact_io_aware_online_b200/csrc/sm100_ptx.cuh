@@ -19,6 +19,32 @@ constexpr unsigned int kStatusMisaligned = 2u;  // dynamic shared memory not 102
 // About two seconds: long enough for any legitimate wait, short enough that a
 // protocol bug ends the kernel instead of hanging the GPU.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Limit of the protocol waits (one role waiting for another), kWaitLimitNs
+// unless a test shortens it through fa_debug_set_wait_limit.  The waits of a
+// role for its own copies and tensor-core operations before the CTA exits
+// always use kWaitLimitNs.
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+// Test hook (fa_debug_set_stall): when nonzero, the producers never issue the
+// first load that the other roles wait for (K/V in the backward, Q in the
+// forward), so those waits run out and the abort path is taken.
+__device__ int g_debug_stall;
+
+// Phase timestamps for performance analysis: compiled out unless FA_TRACE is
+// defined, in which case the first kTraceCtas CTAs of a launch record clock64()
+// at the marked points of each role and iteration.
+#ifdef FA_TRACE
+constexpr int kTraceCtas = 8, kTraceRoles = 8, kTraceIters = 128, kTraceEvents = 4;
+__device__ long long g_trace[8][8][128][4];  // [kTraceCtas][kTraceRoles][kTraceIters][kTraceEvents]
+#define FA_TRACE_AT(role, it, ev)                                            \
+  do {                                                                       \
+    if (blockIdx.x < ::fa::kTraceCtas && (it) < ::fa::kTraceIters)           \
+      ::fa::g_trace[blockIdx.x][role][it][ev] = clock64();                   \
+  } while (0)
+#else
+#define FA_TRACE_AT(role, it, ev) \
+  do {                            \
+  } while (0)
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -57,21 +83,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, or at once when another role of the CTA has already given up
-// (*abort != 0): records the timeout in g_status, raises *abort, returns false.
+// g_wait_limit_ns, or at once when another role of the CTA has already given
+// up (*abort != 0): records the timeout in g_status, raises *abort, returns
+// false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
+  const unsigned long long limit = *static_cast<volatile unsigned long long*>(&g_wait_limit_ns);
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit) {
       atomicOr(&g_status, kStatusTimeout);
       *abort = 1;
       return false;
+    }
+  }
+}
+
+// Waits (at most kWaitLimitNs, whatever the abort flag says) for a phase that
+// is sure to complete: a role's own copies or tensor-core operations, drained
+// before the CTA exits.  Records a timeout if it ever gives up.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      atomicOr(&g_status, kStatusTimeout);
+      return;
     }
   }
 }
@@ -133,7 +175,19 @@ __device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, bool four
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until at most N committed bulk groups of this thread still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Element-wise fp32 add of `bytes` of shared memory into global memory, done by
+// the TMA unit (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
 // Makes generic-proxy shared-memory writes visible to the async proxy (TMA, UMMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -157,6 +211,18 @@ __device__ __forceinline__ void regs_inc() {
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also ANDs a predicate over the participating threads, so
+// that they all take the same branch afterwards.
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -283,6 +349,11 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t r;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
   return r;
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

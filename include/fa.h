@@ -33,6 +33,9 @@
  *  stream    a cudaStream_t passed as void*; NULL means the legacy default
  *            stream.  Every call only enqueues work and returns without
  *            synchronising; results are ready when the stream reaches them.
+ *            The kernels run on the current device (cudaSetDevice), which must
+ *            be the stream's device and own every pointer; a stream of another
+ *            device is rejected with FA_ERR_INVALID_ARG.
  *  Errors    argument errors are detected on the host before anything is
  *            enqueued and leave all buffers untouched; a failed launch returns
  *            FA_ERR_CUDA.  A device-side bounded wait that gives up (after about
@@ -297,6 +300,28 @@ fa_status fa_last_device_status(void* stream);
  * to switch it off.  Process-wide and not thread-safe.
  */
 void fa_set_timing_events(void* start, void* stop);
+
+/*
+ * Test hooks for the failure-detection path (not for production use; both are
+ * process-wide, per device, and take effect for kernels launched afterwards).
+ *
+ * fa_debug_set_wait_limit: the limit, in nanoseconds, after which a kernel's
+ *   wait for another role of its CTA (a tile load, a tensor-core product, a
+ *   softmax step) gives up; 0 restores the default of about two seconds.  A
+ *   CTA whose wait gives up records FA_ERR_TIMEOUT in the device status word,
+ *   stops its other roles, waits (always with the default limit) for its own
+ *   copies and tensor-core operations in flight, frees its tensor memory and
+ *   returns; the outputs of that call are then undefined.
+ * fa_debug_set_stall: while nonzero, the sm_100a kernels never issue their
+ *   first tile load (K/V in the backward, Q in the forward), so every CTA's
+ *   waits for it run out and the call reports FA_ERR_TIMEOUT through
+ *   fa_last_device_status(); 0 restores normal operation.  The fp32 path has
+ *   no waits and ignores it.
+ * Both synchronise with the device (cudaMemcpyToSymbol on the legacy stream)
+ * and return FA_ERR_CUDA if that fails.
+ */
+fa_status fa_debug_set_wait_limit(unsigned long long ns);
+fa_status fa_debug_set_stall(int on);
 
 /* Static, NUL-terminated description of a status code. */
 const char* fa_status_string(fa_status s);

@@ -3,7 +3,8 @@ the same seeded inputs.
 
 Small cases cover every output element and span several tiles plus a ragged
 tail; the full-size workloads run in the launch configuration the benchmark
-times and are compared on whole sampled heads (whole GQA groups).
+times and are compared on whole sampled heads (whole GQA groups), and on every
+head for the two workloads whose oracle takes about a minute.
 """
 import time
 
@@ -93,6 +94,22 @@ def test_full_workload_sampled_heads(name):
     secs = time.perf_counter() - t0
     worst = check_groups(w, got, want)
     print(name, worst, f"oracle {secs:.1f} s for {len(FULL[name])} kv group(s)")
+
+
+@pytest.mark.parametrize("name", ["bf16_b4h16_n2048_d64", "bf16_causal_b2h16_n8192_d128"])
+def test_full_workload_every_head(name):
+    """Every head of the two workloads the oracle finishes in about a minute:
+    a fault confined to some heads (the grid's head grouping, the dQ
+    accumulator's addressing) cannot hide between sampled heads."""
+    w = W.WORKLOADS[name]
+    x = W.make_inputs(w)
+    got = gpu_run(w, x)
+    t0 = time.perf_counter()
+    worst = {}
+    for grp in _all_groups(w):  # one kv group at a time keeps the oracle's memory small
+        for k_, e in check_groups(w, got, oracle_groups(w, x, [grp])).items():
+            worst[k_] = max(worst.get(k_, 0.0), e)
+    print(name, worst, f"oracle {time.perf_counter() - t0:.1f} s for all {w.B * w.H} heads")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
