@@ -24,13 +24,10 @@
 //   warps 4-7   the same for query columns 64-127
 //   warps 8-11  dQ drain (one thread per query row of the dQ tile) and the
 //               final dK/dV epilogue (one thread per key row)
-//   warp 12     tcgen05.mma issuer, stream A (S^T, dV) and TMEM owner
+//   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
 //   warp 13     TMA producer of the Q tiles and their LSE / D rows
-//   warp 14     tcgen05.mma issuer, stream B (dP^T, dK, dQ)
+//   warp 14     idle (completes the fourth warpgroup)
 //   warp 15     TMA producer of the dO tiles
-// The two MMA streams touch disjoint TMEM regions (A: S^T and dV; B: dP^T, dK
-// and dQ), so each keeps its own order and a thread blocked pushing one
-// stream's instructions into a full tensor-core queue never delays the other.
 // Registers: 128 per thread at launch; the fourth warpgroup drops to 64, the
 // compute warpgroups rise to 144 and the drain to 160 (144 + 144 + 160 + 64 =
 // 4 * 128), so a drain thread holds a whole dQ row and releases the TMEM tile
@@ -111,9 +108,9 @@ struct BwdCfg {
   static constexpr int kDqChunkBytes = 128 * 32 * 4;     // 32 fp32 columns of a 128-row dQ tile
   static constexpr int kDqChunks = D / 32;               // chunks per dQ tile
   static constexpr int kDqStages = 2;                    // staging buffers of the dQ reduction
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDoStages + 11;
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDoStages + 10;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: at D = 128 this is 231,584 of the
+  // so no alignment slack is reserved: at D = 128 this is 231,576 of the
   // 232,448 bytes a CTA may use.
   static constexpr int kSmemBytes = 2 * kTileBytes + kQStages * kTileBytes + kDoStages * kTileBytes + kDsBytes +
                                     kDqStages * kDqChunkBytes + kQStages * kVecBytes + 8 * kNumBars + 16;
@@ -306,8 +303,7 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* dq_empty = s_full + 5;
   uint64_t* kv_done = s_full + 6;
   uint64_t* epi_bar = s_full + 7;
-  uint64_t* a_idle = s_full + 8;  // stream A: every product it issued has completed
-  uint64_t* b_idle = s_full + 9;  // stream B: the same
+  uint64_t* mma_idle = s_full + 8;  // every product the MMA thread issued has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -369,11 +365,11 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(kv_full, 1);
     for (int i = 0; i < C::kQStages; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 2);  // one commit from each MMA stream
+      mbar_init(&q_empty[i], 1);
     }
     for (int i = 0; i < C::kDoStages; ++i) {
       mbar_init(&do_full[i], 1);
-      mbar_init(&do_empty[i], 2);  // dP^T (stream B) and dV (stream A) have read it
+      mbar_init(&do_empty[i], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -381,10 +377,9 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
-    mbar_init(kv_done, 2);  // dV (stream A) and dK (stream B) complete
+    mbar_init(kv_done, 1);  // dV and dK complete
     mbar_init(epi_bar, 128);
-    mbar_init(a_idle, 1);
-    mbar_init(b_idle, 1);
+    mbar_init(mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -396,7 +391,14 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) FA_TRACE_AT(6, 0, 0);
+  if (threadIdx.x == 0) {
+    FA_TRACE_AT(6, 0, 0);
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    FA_TRACE_CTA(0, smid);
+    FA_TRACE_CTA(1, total);
+    FA_TRACE_CTA(2, globaltimer_ns());
+  }
 
   if (warp >= 12) {
     regs_dec<64>();
@@ -470,8 +472,13 @@ __global__ void __launch_bounds__(512, 1)
       }
       for (int s = 0; s < C::kDoStages; ++s)
         if (issued[s] > 0) mbar_wait_drain(&do_full[s], (issued[s] - 1) & 1);
-    } else if ((warp == 12 || warp == 14) && lane == 0) {
-      // ---------------------------------------------------------- MMA issuers
+    } else if (warp == 12 && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      // One thread issues every product in a fixed order, so that the tensor
+      // pipe works on the critical chain first:
+      //   ... dK_i, dQ_i, [dQ_i drained] dP^T_{i+1}, [P_{i+1} ready] dV_{i+1}, S^T_{i+2}, ...
+      // dV and the next S^T then run while the compute warps form dS, and the
+      // next dP^T is never queued behind them.
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
                      aDS = smem_u32(sDS);
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
@@ -495,79 +502,64 @@ __global__ void __launch_bounds__(512, 1)
                   sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
       };
       bool ok = mbar_wait(kv_full, 0, abort_flag);
-      if (warp == 12) {
-        // stream A: S^T_i = K Q_i^T, then dV += P_i^T dO_i once P_i is in TMEM
-        if (ok && total > 0 && (ok = mbar_wait(&q_full[0], 0, abort_flag))) {
-          tc_fence_after();
-          kmajor_nt(C::kColS, aK, st_q(0));
-          umma_commit(s_full);
-        }
-        for (int it = 0; ok && it < total; ++it) {
-          const int s = it % C::kQStages, s1 = (it + 1) % C::kQStages, so = it % C::kDoStages;
-          if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
-          FA_TRACE_AT(2, it, 0);
-          if (!(ok = mbar_wait(&do_full[so], (it / C::kDoStages) & 1, abort_flag))) break;
-          tc_fence_after();
-          ts_acc(C::kColDV, C::kColS, st_do(so), it > 0);  // dV += P^T dO
-          umma_commit(&do_empty[so]);
-          umma_commit(&q_empty[s]);  // S^T of this tile (issued earlier) has read Q
-          FA_TRACE_AT(2, it, 1);
-          if (it + 1 < total) {
-            if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kQStages) & 1, abort_flag))) break;
-            FA_TRACE_AT(2, it, 2);
-            tc_fence_after();
-            kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
-            umma_commit(s_full);
-            FA_TRACE_AT(2, it, 3);
-          }
-        }
-        if (ok) umma_commit(kv_done);
-        // Before the CTA frees TMEM: every product this thread issued has completed.
-        umma_commit(a_idle);
-        mbar_wait_drain(a_idle, 0);
-      } else {
-        // stream B: dP^T_i = V dO_i^T; once dS_i is ready dK += dS_i^T Q_i and dQ_i = dS_i K
-        if (ok && total > 0 && (ok = mbar_wait(&do_full[0], 0, abort_flag))) {
-          tc_fence_after();
-          kmajor_nt(C::kColDP, aV, st_do(0));
-          umma_commit(dp_full);
-          umma_commit(&do_empty[0]);
-        }
-        for (int it = 0; ok && it < total; ++it) {
-          const int s = it % C::kQStages, so1 = (it + 1) % C::kDoStages;
-          if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
-          FA_TRACE_AT(3, it, 0);
-          if (!(ok = mbar_wait(&q_full[s], (it / C::kQStages) & 1, abort_flag))) break;
-          tc_fence_after();
-          ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
-          if (!C::kAliasDq && it > 0) {
-            if (!(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag))) break;
-            tc_fence_after();
-          }
-#pragma unroll
-          for (int k = 0; k < 8; ++k)  // dQ_i = dS K (both operands MN-major in smem)
-            umma_ss(tmem + C::kColDQ, sdesc_sw128(aDS + k * 2048, 16384, 1024),
-                    sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
-          umma_commit(dq_full);
-          umma_commit(&q_empty[s]);
-          FA_TRACE_AT(3, it, 1);
-          if (it + 1 < total) {
-            if (C::kAliasDq) {
-              if (!(ok = mbar_wait(dq_empty, it & 1, abort_flag))) break;
-            }
-            if (!(ok = mbar_wait(&do_full[so1], ((it + 1) / C::kDoStages) & 1, abort_flag))) break;
-            FA_TRACE_AT(3, it, 2);
-            tc_fence_after();
-            kmajor_nt(C::kColDP, aV, st_do(so1));  // dP^T of the next query tile
-            umma_commit(dp_full);
-            umma_commit(&do_empty[so1]);
-            FA_TRACE_AT(3, it, 3);
-          }
-        }
-        if (ok) umma_commit(kv_done);
-        umma_commit(b_idle);
-        mbar_wait_drain(b_idle, 0);
+      if (ok && total > 0 && (ok = mbar_wait(&q_full[0], 0, abort_flag))) {
+        tc_fence_after();
+        kmajor_nt(C::kColS, aK, st_q(0));  // S^T_0 = K Q_0^T
+        umma_commit(s_full);
       }
+      if (ok && total > 0 && (ok = mbar_wait(&do_full[0], 0, abort_flag))) {
+        tc_fence_after();
+        kmajor_nt(C::kColDP, aV, st_do(0));  // dP^T_0 = V dO_0^T
+        umma_commit(dp_full);
+      }
+      for (int it = 0; ok && it < total; ++it) {
+        const int s = it % C::kQStages, s1 = (it + 1) % C::kQStages;
+        const int so = it % C::kDoStages, so1 = (it + 1) % C::kDoStages;
+        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
+        FA_TRACE_AT(2, it, 0);
+        tc_fence_after();
+        ts_acc(C::kColDV, C::kColS, st_do(so), it > 0);  // dV += P^T dO (dO_i landed before dP^T_i)
+        umma_commit(&do_empty[so]);                       // dP^T_i and dV_i have read dO_i
+        FA_TRACE_AT(2, it, 1);
+        if (it + 1 < total) {
+          if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kQStages) & 1, abort_flag))) break;
+          FA_TRACE_AT(2, it, 2);
+          tc_fence_after();
+          kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
+          umma_commit(s_full);
+          FA_TRACE_AT(2, it, 3);
+        }
+        if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
+        FA_TRACE_AT(3, it, 0);
+        tc_fence_after();
+        ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
+        if (!C::kAliasDq && it > 0) {
+          if (!(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)  // dQ_i = dS K (both operands MN-major in smem)
+          umma_ss(tmem + C::kColDQ, sdesc_sw128(aDS + k * 2048, 16384, 1024),
+                  sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
+        umma_commit(dq_full);
+        umma_commit(&q_empty[s]);
+        FA_TRACE_AT(3, it, 1);
+        if (it + 1 < total) {
+          if (C::kAliasDq) {  // the dQ tile shares the dP^T columns
+            if (!(ok = mbar_wait(dq_empty, it & 1, abort_flag))) break;
+          }
+          if (!(ok = mbar_wait(&do_full[so1], ((it + 1) / C::kDoStages) & 1, abort_flag))) break;
+          FA_TRACE_AT(3, it, 2);
+          tc_fence_after();
+          kmajor_nt(C::kColDP, aV, st_do(so1));  // dP^T of the next query tile
+          umma_commit(dp_full);
+          FA_TRACE_AT(3, it, 3);
+        }
+      }
+      if (ok) umma_commit(kv_done);
+      // Before the CTA frees TMEM: every product this thread issued has completed.
+      umma_commit(mma_idle);
+      mbar_wait_drain(mma_idle, 0);
     }
     __syncwarp();
   } else if (warp < 8) {
@@ -761,7 +753,10 @@ __global__ void __launch_bounds__(512, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0) FA_TRACE_AT(6, 0, 1);
+  if (threadIdx.x == 0) {
+    FA_TRACE_AT(6, 0, 1);
+    FA_TRACE_CTA(3, globaltimer_ns());
+  }
   if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);

@@ -872,6 +872,10 @@ int fa_trace_read(void* dst, size_t bytes) {
   if (bytes > kTraceBytes) bytes = kTraceBytes;
   return cudaMemcpyFromSymbol(dst, fa::g_trace, bytes) == cudaSuccess ? 0 : 1;
 }
+int fa_trace_cta_read(void* dst, size_t bytes) {
+  if (bytes > sizeof(long long) * 16384 * 4) bytes = sizeof(long long) * 16384 * 4;
+  return cudaMemcpyFromSymbol(dst, fa::g_trace_cta, bytes) == cudaSuccess ? 0 : 1;
+}
 int fa_trace_clear(void) {
   static long long zero[kTraceBytes / sizeof(long long)];
   return cudaMemcpyToSymbol(fa::g_trace, zero, sizeof(zero)) == cudaSuccess ? 0 : 1;

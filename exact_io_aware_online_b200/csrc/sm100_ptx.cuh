@@ -40,9 +40,19 @@ __device__ long long g_trace[8][8][128][4];  // [kTraceCtas][kTraceRoles][kTrace
     if (blockIdx.x < ::fa::kTraceCtas && (it) < ::fa::kTraceIters)           \
       ::fa::g_trace[blockIdx.x][role][it][ev] = clock64();                   \
   } while (0)
+// Per-CTA record of every CTA of a launch: SM id, iteration count, start and
+// end (%globaltimer, ns).
+__device__ long long g_trace_cta[16384][4];
+#define FA_TRACE_CTA(ev, val)                                                          \
+  do {                                                                                 \
+    if (blockIdx.x < 16384) ::fa::g_trace_cta[blockIdx.x][ev] = static_cast<long long>(val); \
+  } while (0)
 #else
 #define FA_TRACE_AT(role, it, ev) \
   do {                            \
+  } while (0)
+#define FA_TRACE_CTA(ev, val) \
+  do {                        \
   } while (0)
 #endif
 
