@@ -11,27 +11,28 @@
 // Three kernels run on one stream:
 //   bwd_pre_kernel   -D_i, -LSE_i * log2(e) (-inf on padding rows) and a
 //                    zeroed fp32 dQ accumulator, all in the caller's workspace;
-//   bwd_sm100_kernel one CTA per (batch, kv head, 128-key tile): K_j and V_j
-//                    stay in shared memory while the CTA walks every query
-//                    tile (of every query head of the GQA group) that can see
-//                    them; dK_j and dV_j accumulate in TMEM and are written
-//                    once, dQ partial tiles are added into the accumulator;
+//   bwd_sm100_kernel one CTA per (batch, kv head, pair of 128-key tiles): for
+//                    each tile j, K_j and V_j stay in shared memory while the
+//                    CTA walks every query tile (of every query head of the
+//                    GQA group) that can see them; dK_j and dV_j accumulate in
+//                    TMEM and are written once, dQ partial tiles are added
+//                    into the accumulator;
 //   bwd_dq_kernel    dQ = bf16(scale * accumulator).
 //
 // Main-kernel roles (512 threads, four warpgroups):
 //   warps 0-3   P / dS for query columns 0-63 of the tile, one thread per key
 //               row (TMEM lanes 0-127)
 //   warps 4-7   the same for query columns 64-127
-//   warps 8-11  dQ drain (one thread per query row of the dQ tile) and the
-//               final dK/dV epilogue (one thread per key row)
+//   warps 8-11  dQ drain (one thread per query row of the dQ tile) and each
+//               tile's dK/dV epilogue (one thread per key row)
 //   warp 12     tcgen05.mma issuer (one thread) and TMEM owner
 //   warp 13     TMA producer of the Q tiles and their LSE / D rows
 //   warp 14     idle (completes the fourth warpgroup)
 //   warp 15     TMA producer of the dO tiles
-// Registers: 128 per thread at launch; the fourth warpgroup drops to 64, the
-// compute warpgroups rise to 144 and the drain to 160 (144 + 144 + 160 + 64 =
-// 4 * 128), so a drain thread holds a whole dQ row and releases the TMEM tile
-// at once.
+// Registers: 128 per thread at launch; the fourth warpgroup drops to 96, the
+// compute warpgroups rise to 136 and the drain to 144 (136 + 136 + 144 + 96 =
+// 4 * 128, checked below), so a drain thread holds a whole dQ row and releases
+// the TMEM tile at once.
 //
 // dQ reduction.  Every (key tile, query tile) pair adds a 128 x D fp32 partial
 // into the global accumulator.  The drain loads the partial from TMEM into
@@ -73,6 +74,8 @@ struct BwdParams {
   int causal, window;
   int ntiles;  // Np / 128
   int group;   // kv heads per rasterisation group (kept L2-resident together)
+  int slots;   // CTAs per kv head: ceil(ntiles / 2), each running up to two key tiles
+  int pairs;   // 1: a CTA runs key tiles j and ntiles - 1 - j (causal); 0: tiles 2j and 2j + 1
   // block-sparse mode (non-null bmask): 0/1 per 128 x 128 block, [query block]
   // [key block] per query head, bmask_hs elements apart (0: shared by all heads)
   const uint8_t* bmask;
@@ -108,9 +111,9 @@ struct BwdCfg {
   static constexpr int kDqChunkBytes = 128 * 32 * 4;     // 32 fp32 columns of a 128-row dQ tile
   static constexpr int kDqChunks = D / 32;               // chunks per dQ tile
   static constexpr int kDqStages = 2;                    // staging buffers of the dQ reduction
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDoStages + 10;
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDoStages + 11;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: at D = 128 this is 231,576 of the
+  // so no alignment slack is reserved: at D = 128 this is 231,584 of the
   // 232,448 bytes a CTA may use.
   static constexpr int kSmemBytes = 2 * kTileBytes + kQStages * kTileBytes + kDoStages * kTileBytes + kDsBytes +
                                     kDqStages * kDqChunkBytes + kQStages * kVecBytes + 8 * kNumBars + 16;
@@ -120,6 +123,11 @@ struct BwdCfg {
   static constexpr uint32_t kColDQ = kAliasDq ? 128 : 256 + 2 * D;
 };
 static_assert(BwdCfg<128>::kSmemBytes <= 232448, "backward shared memory over the per-CTA limit");
+// Per-thread register budgets after setmaxnreg (compute, compute, drain, MMA +
+// producers): an increase waits until decreases have freed the registers, so
+// the four must add up to the 4 x 128 the 512-thread launch provides.
+constexpr int kBwdRegsCompute = 136, kBwdRegsDrain = 144, kBwdRegsOther = 96;
+static_assert(2 * kBwdRegsCompute + kBwdRegsDrain + kBwdRegsOther == 4 * 128, "register split must sum to the launch");
 
 // ---------------------------------------------------------------- preprocess
 // Half a warp per row (16 lanes x 16 bytes of O and of dO for D = 128, two rows
@@ -270,6 +278,14 @@ __device__ __forceinline__ void exp_cols64(float (&x)[64], const float* nLv, flo
 }
 
 // ---------------------------------------------------------------- main kernel
+// Work units are (kv head, 128-key tile) pairs; each CTA runs up to two units
+// of one kv head back to back, its pipelines running on from the first unit
+// into the second.  Under a causal mask the two are key tiles j and
+// ntiles - 1 - j, whose query-tile counts add up to the same total for every
+// CTA, so the grid has no long and short CTAs; otherwise they are adjacent
+// tiles (which share most of their query tiles in a window band).
+constexpr int kBwdMaxUnits = 2;
+
 template <int D, bool kMask, bool kStrided = false>
 __global__ void __launch_bounds__(512, 1)
     bwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -287,7 +303,7 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sQ = smem_raw + 2 * C::kTileBytes;              // Q stage s at s * kTileBytes
   uint8_t* sDO = sQ + C::kQStages * C::kTileBytes;        // dO stage s at s * kTileBytes
   uint8_t* sDS = sDO + C::kDoStages * C::kTileBytes;
-  uint8_t* sDQ = sDS + C::kDsBytes;                        // dQ staging buffers, kDqChunkBytes each
+  uint8_t* sDQ = sDS + C::kDsBytes;  // dQ staging buffers, kDqChunkBytes each; dK/dV epilogue staging
   uint8_t* sVec = sDQ + C::kDqStages * C::kDqChunkBytes;  // Q stage s: -LSE*log2(e) [128] then -D [128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sVec + C::kQStages * C::kVecBytes);
   uint64_t* kv_full = bars;
@@ -301,65 +317,76 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* ds_full = s_full + 3;
   uint64_t* dq_full = s_full + 4;
   uint64_t* dq_empty = s_full + 5;
-  uint64_t* kv_done = s_full + 6;
-  uint64_t* epi_bar = s_full + 7;
-  uint64_t* mma_idle = s_full + 8;  // every product the MMA thread issued has completed
+  uint64_t* kv_done = s_full + 6;    // a unit's dV and dK are complete in TMEM
+  uint64_t* kv_empty = s_full + 7;   // a unit's products no longer read K and V
+  uint64_t* acc_empty = s_full + 8;  // a unit's dV and dK have been read out of TMEM
+  uint64_t* mma_idle = s_full + 9;   // every product the MMA thread issued has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work unit: key tile j of kv head bkv.  Groups of p.group kv heads run
-  // together (their Q, dO, K, V and dQ accumulator stay in L2); inside a group
-  // the smallest j (the most query tiles under a causal mask) goes first.
+  // ---- this CTA's kv head and slot.  Groups of p.group kv heads run together
+  // (their Q, dO, K, V and dQ accumulator stay in L2).
   const int BHkv = p.B * p.Hkv;
-  const int per_group = p.group * p.ntiles;
+  const int per_group = p.group * p.slots;
   const int grp = static_cast<int>(blockIdx.x) / per_group;
   const int g0 = grp * p.group;
   const int gsz = min(p.group, BHkv - g0);
   const int rem = static_cast<int>(blockIdx.x) - grp * per_group;
-  const int j = rem / gsz;
+  const int slot = rem / gsz;
   const int bkv = g0 + rem % gsz;
   const int b = bkv / p.Hkv, kh = bkv % p.Hkv;
-  const int k0 = j * 128;
   const int Lb = valid_rows(p, b);
-  int ilo = 0, ihi = (max(Lb, 1) - 1) / 128;  // query tiles holding valid rows
-  if (p.causal) ilo = j;
-  if (p.window >= 0) {
-    ilo = max(ilo, max(0, k0 - p.window) / 128);
-    ihi = min(ihi, (k0 + 127 + p.window) / 128);
-  }
-  // Work list: (query head hq of the group, query tile i) pairs in increasing
-  // order, skipping blocks a block-sparse mask switches off.  Every role walks
-  // it with its own QCursor, so all roles see the same sequence.
+  const int bh0 = b * p.H + kh * p.g;  // first query head of the GQA group
+  const int nunits = p.pairs ? (p.ntiles - 1 - slot != slot ? 2 : 1) : (2 * slot + 1 < p.ntiles ? 2 : 1);
+  // One unit: key tile j, its query-tile range [ilo, ihi] and the number of
+  // (query head, query tile) work items.  Work items are walked in increasing
+  // order, skipping blocks a block-sparse mask switches off; every role walks
+  // them with its own cursor, so all roles see the same sequence.
   // (kMask: the block-sparse variant; the dense kernels compile no mask test.)
-  const int bh0 = b * p.H + kh * p.g;
-  auto active = [&](int hq, int i) {
-    return !kMask || p.bmask[(bh0 + hq) * p.bmask_hs + static_cast<long long>(i) * p.ntiles + j] != 0;
+  struct Unit {
+    int j, k0, ilo, ihi, total;
   };
   struct QCursor {
     int hq, i;
   };
-  auto advance = [&](QCursor c) {  // next active pair strictly after c
+  auto active = [&](const Unit& U, int hq, int i) {
+    return !kMask || p.bmask[(bh0 + hq) * p.bmask_hs + static_cast<long long>(i) * p.ntiles + U.j] != 0;
+  };
+  auto advance = [&](const Unit& U, QCursor c) {  // next active item strictly after c
     do {
-      if (++c.i > ihi) {
-        c.i = ilo;
+      if (++c.i > U.ihi) {
+        c.i = U.ilo;
         ++c.hq;
       }
-    } while (kMask && c.hq < p.g && !active(c.hq, c.i));
+    } while (kMask && c.hq < p.g && !active(U, c.hq, c.i));
     return c;
   };
-  auto first = [&]() {
-    QCursor c{0, ilo};
-    if (kMask && !active(0, ilo)) c = advance(c);
+  auto first = [&](const Unit& U) {
+    QCursor c{0, U.ilo};
+    if (kMask && !active(U, 0, U.ilo)) c = advance(U, c);
     return c;
   };
-  const bool no_work = ilo > ihi || k0 >= Lb;  // nothing reaches this key tile
-  int total = no_work ? 0 : (ihi - ilo + 1) * p.g;
-  if (kMask && !no_work) {
-    total = 0;
-    for (QCursor c = first(); c.hq < p.g; c = advance(c)) ++total;
-  }
+  auto unit = [&](int u) {
+    Unit U;
+    U.j = p.pairs ? (u == 0 ? slot : p.ntiles - 1 - slot) : 2 * slot + u;
+    U.k0 = U.j * 128;
+    U.ilo = 0;
+    U.ihi = (max(Lb, 1) - 1) / 128;  // query tiles holding valid rows
+    if (p.causal) U.ilo = U.j;
+    if (p.window >= 0) {
+      U.ilo = max(U.ilo, max(0, U.k0 - p.window) / 128);
+      U.ihi = min(U.ihi, (U.k0 + 127 + p.window) / 128);
+    }
+    const bool no_work = U.ilo > U.ihi || U.k0 >= Lb;  // nothing reaches this key tile
+    U.total = no_work ? 0 : (U.ihi - U.ilo + 1) * p.g;
+    if (kMask && !no_work) {
+      U.total = 0;
+      for (QCursor c = first(U); c.hq < p.g; c = advance(U, c)) ++U.total;
+    }
+    return U;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -377,8 +404,9 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(ds_full, 256);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
-    mbar_init(kv_done, 1);  // dV and dK complete
-    mbar_init(epi_bar, 128);
+    mbar_init(kv_done, 1);
+    mbar_init(kv_empty, 1);
+    mbar_init(acc_empty, 128);
     mbar_init(mma_idle, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -395,56 +423,66 @@ __global__ void __launch_bounds__(512, 1)
     FA_TRACE_AT(6, 0, 0);
     uint32_t smid;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    int items = 0;
+    for (int u = 0; u < nunits; ++u) items += unit(u).total;
     FA_TRACE_CTA(0, smid);
-    FA_TRACE_CTA(1, total);
+    FA_TRACE_CTA(1, items);
     FA_TRACE_CTA(2, globaltimer_ns());
   }
 
   if (warp >= 12) {
-    regs_dec<64>();
+    regs_dec<kBwdRegsOther>();
     if (warp == 13 && lane == 0) {
-      // ---------------------------------------------------------- producer: K, V, then Q + LSE + D
+      // ---------------------------------------------------------- producer: K, V, Q + LSE + D
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const bool stall = g_debug_stall != 0;  // test hook: K/V never arrive
-      if (!stall) {
-        mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
-        for (int c = 0; c < C::kChunks; ++c) {
-          if constexpr (kStrided) {
-            tma_load_tile(&tmK, p.map4 & kBMapK, kv_full, sK + c * 16384, c * 64, k0, bkv, kh, b);
-            tma_load_tile(&tmV, p.map4 & kBMapV, kv_full, sV + c * 16384, c * 64, k0, bkv, kh, b);
-          } else {
-            tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, k0, bkv);
-            tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, k0, bkv);
-          }
-        }
-      }
+      const bool stall = g_debug_stall != 0;  // test hook: the first K/V never arrive
       int issued[C::kQStages];
 #pragma unroll
       for (int i = 0; i < C::kQStages; ++i) issued[i] = 0;
-      QCursor cur = first();
-      for (int it = 0; it < total; ++it, cur = advance(cur)) {
-        const int s = it % C::kQStages;
-        if (!mbar_wait(&q_empty[s], ((it / C::kQStages) & 1) ^ 1, abort_flag)) break;
-        FA_TRACE_AT(5, it, 0);
-        mbar_arrive_expect_tx(&q_full[s], C::kTileBytes + C::kVecBytes);
-        const int row0 = cur.i * 128, bh = bh0 + cur.hq;
-        uint8_t* st = sQ + s * C::kTileBytes;
-        for (int c = 0; c < C::kChunks; ++c) {
-          if constexpr (kStrided)
-            tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, row0, bh, kh * p.g + cur.hq,
-                          b);
-          else
-            tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
+      int kv_loaded = 0, git = 0;
+      bool ok = true;
+      for (int u = 0; ok && u < nunits; ++u) {
+        const Unit U = unit(u);
+        // K and V of this unit replace the previous unit's once its products are done with them
+        if (u > 0 && !(ok = mbar_wait(kv_empty, (u - 1) & 1, abort_flag))) break;
+        if (!(stall && u == 0)) {
+          mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+          for (int c = 0; c < C::kChunks; ++c) {
+            if constexpr (kStrided) {
+              tma_load_tile(&tmK, p.map4 & kBMapK, kv_full, sK + c * 16384, c * 64, U.k0, bkv, kh, b);
+              tma_load_tile(&tmV, p.map4 & kBMapV, kv_full, sV + c * 16384, c * 64, U.k0, bkv, kh, b);
+            } else {
+              tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, U.k0, bkv);
+              tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, U.k0, bkv);
+            }
+          }
+          kv_loaded = u + 1;
         }
-        const size_t vrow = static_cast<size_t>(bh) * p.Np + row0;
-        bulk_load(sVec + s * C::kVecBytes, p.nlse2 + vrow, 512, &q_full[s]);
-        bulk_load(sVec + s * C::kVecBytes + 512, p.nD + vrow, 512, &q_full[s]);
-        ++issued[s];
+        QCursor cur = first(U);
+        for (int it = 0; it < U.total; ++it, ++git, cur = advance(U, cur)) {
+          const int s = git % C::kQStages;
+          if (!(ok = mbar_wait(&q_empty[s], ((git / C::kQStages) & 1) ^ 1, abort_flag))) break;
+          FA_TRACE_AT(5, git, 0);
+          mbar_arrive_expect_tx(&q_full[s], C::kTileBytes + C::kVecBytes);
+          const int row0 = cur.i * 128, bh = bh0 + cur.hq;
+          uint8_t* st = sQ + s * C::kTileBytes;
+          for (int c = 0; c < C::kChunks; ++c) {
+            if constexpr (kStrided)
+              tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, row0, bh,
+                            kh * p.g + cur.hq, b);
+            else
+              tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
+          }
+          const size_t vrow = static_cast<size_t>(bh) * p.Np + row0;
+          bulk_load(sVec + s * C::kVecBytes, p.nlse2 + vrow, 512, &q_full[s]);
+          bulk_load(sVec + s * C::kVecBytes + 512, p.nD + vrow, 512, &q_full[s]);
+          ++issued[s];
+        }
       }
       // Never leave the CTA with copies still landing in shared memory.
-      if (!stall) mbar_wait_drain(kv_full, 0);
+      if (kv_loaded > 0) mbar_wait_drain(kv_full, (kv_loaded - 1) & 1);
       for (int s = 0; s < C::kQStages; ++s)
         if (issued[s] > 0) mbar_wait_drain(&q_full[s], (issued[s] - 1) & 1);
     } else if (warp == 15 && lane == 0) {
@@ -453,22 +491,27 @@ __global__ void __launch_bounds__(512, 1)
       int issued[C::kDoStages];
 #pragma unroll
       for (int i = 0; i < C::kDoStages; ++i) issued[i] = 0;
-      QCursor cur = first();
-      for (int it = 0; it < total; ++it, cur = advance(cur)) {
-        const int s = it % C::kDoStages;
-        if (!mbar_wait(&do_empty[s], ((it / C::kDoStages) & 1) ^ 1, abort_flag)) break;
-        FA_TRACE_AT(5, it, 1);
-        mbar_arrive_expect_tx(&do_full[s], C::kTileBytes);
-        const int row0 = cur.i * 128, bh = bh0 + cur.hq;
-        uint8_t* st = sDO + s * C::kTileBytes;
-        for (int c = 0; c < C::kChunks; ++c) {
-          if constexpr (kStrided)
-            tma_load_tile(&tmdO, p.map4 & kBMapDO, &do_full[s], st + c * 16384, c * 64, row0, bh,
-                          kh * p.g + cur.hq, b);
-          else
-            tma_load_3d(&tmdO, &do_full[s], st + c * 16384, c * 64, row0, bh);
+      int git = 0;
+      bool ok = true;
+      for (int u = 0; ok && u < nunits; ++u) {
+        const Unit U = unit(u);
+        QCursor cur = first(U);
+        for (int it = 0; it < U.total; ++it, ++git, cur = advance(U, cur)) {
+          const int s = git % C::kDoStages;
+          if (!(ok = mbar_wait(&do_empty[s], ((git / C::kDoStages) & 1) ^ 1, abort_flag))) break;
+          FA_TRACE_AT(5, git, 1);
+          mbar_arrive_expect_tx(&do_full[s], C::kTileBytes);
+          const int row0 = cur.i * 128, bh = bh0 + cur.hq;
+          uint8_t* st = sDO + s * C::kTileBytes;
+          for (int c = 0; c < C::kChunks; ++c) {
+            if constexpr (kStrided)
+              tma_load_tile(&tmdO, p.map4 & kBMapDO, &do_full[s], st + c * 16384, c * 64, row0, bh,
+                            kh * p.g + cur.hq, b);
+            else
+              tma_load_3d(&tmdO, &do_full[s], st + c * 16384, c * 64, row0, bh);
+          }
+          ++issued[s];
         }
-        ++issued[s];
       }
       for (int s = 0; s < C::kDoStages; ++s)
         if (issued[s] > 0) mbar_wait_drain(&do_full[s], (issued[s] - 1) & 1);
@@ -478,7 +521,8 @@ __global__ void __launch_bounds__(512, 1)
       // pipe works on the critical chain first:
       //   ... dK_i, dQ_i, [dQ_i drained] dP^T_{i+1}, [P_{i+1} ready] dV_{i+1}, S^T_{i+2}, ...
       // dV and the next S^T then run while the compute warps form dS, and the
-      // next dP^T is never queued behind them.
+      // next dP^T is never queued behind them.  The chain runs on from one unit
+      // into the next.
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
                      aDS = smem_u32(sDS);
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
@@ -501,62 +545,83 @@ __global__ void __launch_bounds__(512, 1)
           umma_ts(tmem + dcol, tmem + acol + (k >> 2) * 64 + (k & 3) * 8,
                   sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
       };
-      bool ok = mbar_wait(kv_full, 0, abort_flag);
-      if (ok && total > 0 && (ok = mbar_wait(&q_full[0], 0, abort_flag))) {
-        tc_fence_after();
-        kmajor_nt(C::kColS, aK, st_q(0));  // S^T_0 = K Q_0^T
-        umma_commit(s_full);
-      }
-      if (ok && total > 0 && (ok = mbar_wait(&do_full[0], 0, abort_flag))) {
-        tc_fence_after();
-        kmajor_nt(C::kColDP, aV, st_do(0));  // dP^T_0 = V dO_0^T
-        umma_commit(dp_full);
-      }
-      for (int it = 0; ok && it < total; ++it) {
-        const int s = it % C::kQStages, s1 = (it + 1) % C::kQStages;
-        const int so = it % C::kDoStages, so1 = (it + 1) % C::kDoStages;
-        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
-        FA_TRACE_AT(2, it, 0);
-        tc_fence_after();
-        ts_acc(C::kColDV, C::kColS, st_do(so), it > 0);  // dV += P^T dO (dO_i landed before dP^T_i)
-        umma_commit(&do_empty[so]);                       // dP^T_i and dV_i have read dO_i
-        FA_TRACE_AT(2, it, 1);
-        if (it + 1 < total) {
-          if (!(ok = mbar_wait(&q_full[s1], ((it + 1) / C::kQStages) & 1, abort_flag))) break;
-          FA_TRACE_AT(2, it, 2);
+      bool ok = true;
+      int git = 0;  // work items of the CTA before the current one (barrier phases run on across units)
+      for (int u = 0; ok && u < nunits; ++u) {
+        const Unit U = unit(u);
+        if (!(ok = mbar_wait(kv_full, u & 1, abort_flag))) break;
+        if (U.total > 0) {
+          if (!(ok = mbar_wait(&q_full[git % C::kQStages], (git / C::kQStages) & 1, abort_flag))) break;
           tc_fence_after();
-          kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
+          kmajor_nt(C::kColS, aK, st_q(git % C::kQStages));  // S^T of the first query tile
           umma_commit(s_full);
-          FA_TRACE_AT(2, it, 3);
-        }
-        if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
-        FA_TRACE_AT(3, it, 0);
-        tc_fence_after();
-        ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
-        if (!C::kAliasDq && it > 0) {
-          if (!(ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k)  // dQ_i = dS K (both operands MN-major in smem)
-          umma_ss(tmem + C::kColDQ, sdesc_sw128(aDS + k * 2048, 16384, 1024),
-                  sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
-        umma_commit(dq_full);
-        umma_commit(&q_empty[s]);
-        FA_TRACE_AT(3, it, 1);
-        if (it + 1 < total) {
-          if (C::kAliasDq) {  // the dQ tile shares the dP^T columns
-            if (!(ok = mbar_wait(dq_empty, it & 1, abort_flag))) break;
+          if (C::kAliasDq && git > 0) {  // the previous unit's last dQ tile shares the dP^T columns
+            if (!(ok = mbar_wait(dq_empty, (git - 1) & 1, abort_flag))) break;
           }
-          if (!(ok = mbar_wait(&do_full[so1], ((it + 1) / C::kDoStages) & 1, abort_flag))) break;
-          FA_TRACE_AT(3, it, 2);
+          if (!(ok = mbar_wait(&do_full[git % C::kDoStages], (git / C::kDoStages) & 1, abort_flag))) break;
           tc_fence_after();
-          kmajor_nt(C::kColDP, aV, st_do(so1));  // dP^T of the next query tile
+          kmajor_nt(C::kColDP, aV, st_do(git % C::kDoStages));  // dP^T of the first query tile
           umma_commit(dp_full);
-          FA_TRACE_AT(3, it, 3);
         }
+        for (int it = 0; ok && it < U.total; ++it) {
+          const int g = git + it;
+          const int s = g % C::kQStages, s1 = (g + 1) % C::kQStages;
+          const int so = g % C::kDoStages, so1 = (g + 1) % C::kDoStages;
+          if (!(ok = mbar_wait(p_full, g & 1, abort_flag))) break;
+          if (it == 0 && u > 0) {  // the accumulators start afresh: the previous unit's were read out
+            if (!(ok = mbar_wait(acc_empty, (u - 1) & 1, abort_flag))) break;
+          }
+          FA_TRACE_AT(2, g, 0);
+          tc_fence_after();
+          ts_acc(C::kColDV, C::kColS, st_do(so), it > 0);  // dV += P^T dO (dO_i landed before dP^T_i)
+          umma_commit(&do_empty[so]);                       // dP^T_i and dV_i have read dO_i
+          FA_TRACE_AT(2, g, 1);
+          if (it + 1 < U.total) {
+            if (!(ok = mbar_wait(&q_full[s1], ((g + 1) / C::kQStages) & 1, abort_flag))) break;
+            FA_TRACE_AT(2, g, 2);
+            tc_fence_after();
+            kmajor_nt(C::kColS, aK, st_q(s1));  // S^T of the next query tile
+            umma_commit(s_full);
+            FA_TRACE_AT(2, g, 3);
+          }
+          if (!(ok = mbar_wait(ds_full, g & 1, abort_flag))) break;
+          FA_TRACE_AT(3, g, 0);
+          tc_fence_after();
+          ts_acc(C::kColDK, C::kColDP, st_q(s), it > 0);  // dK += dS^T Q
+          if (!C::kAliasDq && g > 0) {
+            if (!(ok = mbar_wait(dq_empty, (g - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)  // dQ_i = dS K (both operands MN-major in smem)
+            umma_ss(tmem + C::kColDQ, sdesc_sw128(aDS + k * 2048, 16384, 1024),
+                    sdesc_sw128(aK + k * 2048, 16384, 1024), kIdQ, k > 0);
+          umma_commit(dq_full);
+          umma_commit(&q_empty[s]);
+          FA_TRACE_AT(3, g, 1);
+          if (it + 1 < U.total) {
+            if (C::kAliasDq) {  // the dQ tile shares the dP^T columns
+              if (!(ok = mbar_wait(dq_empty, g & 1, abort_flag))) break;
+            }
+            if (!(ok = mbar_wait(&do_full[so1], ((g + 1) / C::kDoStages) & 1, abort_flag))) break;
+            FA_TRACE_AT(3, g, 2);
+            tc_fence_after();
+            kmajor_nt(C::kColDP, aV, st_do(so1));  // dP^T of the next query tile
+            umma_commit(dp_full);
+            FA_TRACE_AT(3, g, 3);
+          }
+        }
+        if (!ok) break;
+        if (U.total == 0 && u > 0) {
+          // A unit without products must still not complete its kv_done phase
+          // before the drain has consumed the previous one (a waiter on a
+          // phase parity must never be overtaken by two phases).
+          if (!(ok = mbar_wait(acc_empty, (u - 1) & 1, abort_flag))) break;
+        }
+        git += U.total;
+        umma_commit(kv_empty);  // K and V may be replaced once these products complete
+        umma_commit(kv_done);   // dV and dK of the unit are complete
       }
-      if (ok) umma_commit(kv_done);
       // Before the CTA frees TMEM: every product this thread issued has completed.
       umma_commit(mma_idle);
       mbar_wait_drain(mma_idle, 0);
@@ -564,192 +629,231 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ P and dS
-    regs_inc<144>();
+    regs_inc<kBwdRegsCompute>();
     // Warpgroup w handles query columns [64w, 64w + 64); one key row per thread.
     const int w = warp >> 2, wl = warp & 3;
     const int r = wl * 32 + lane;
-    const int key = k0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::kColS + 64 * w;
     const uint32_t tDP = tmem + lane_off + C::kColDP + 64 * w;
     const float sl2 = p.scale_log2;
     const int ds_chunk = w;  // 64-column (128-byte) block of the dS tile
-    const bool tile_valid = k0 + 127 < Lb;  // no padded key in this key tile
-    const bool key_valid = key < Lb;
     bool ok = true;
-    QCursor cur = first();
-    for (int it = 0; it < total; ++it, cur = advance(cur)) {
-      const int s = it % C::kQStages;
-      const int q0 = cur.i * 128 + 64 * w;  // first query of my columns
-      const float* nLv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes) + 64 * w;
-      const float* nDv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes + 512) + 64 * w;
-      bool full = tile_valid;  // every (query, key) pair of my 64 columns allowed?
-      if (p.causal) full = full && (k0 + 127 <= q0);
-      if (p.window >= 0) full = full && (q0 + 63 - k0 <= p.window) && (k0 + 127 - q0 <= p.window);
-      // (warp-uniform outcomes: the TMEM loads and stores below are warp-collective)
-      ok = mbar_wait(&q_full[s], (it / C::kQStages) & 1, abort_flag);  // LSE / D landed
-      ok = ok && mbar_wait(s_full, it & 1, abort_flag);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 0);
-      tc_fence_after();
-      float pv[64];  // the fp32 weights P^T of my 64 columns
-      {
-        uint32_t sv[64];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_wait_ld();
+    int git = 0;
+    for (int u = 0; ok && u < nunits; ++u) {
+      const Unit U = unit(u);
+      const int key = U.k0 + r;
+      const bool tile_valid = U.k0 + 127 < Lb;  // no padded key in this key tile
+      const bool key_valid = key < Lb;
+      QCursor cur = first(U);
+      for (int it = 0; it < U.total; ++it, cur = advance(U, cur)) {
+        const int g = git + it;
+        const int s = g % C::kQStages;
+        const int q0 = cur.i * 128 + 64 * w;  // first query of my columns
+        const float* nLv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes) + 64 * w;
+        const float* nDv = reinterpret_cast<const float*>(sVec + s * C::kVecBytes + 512) + 64 * w;
+        bool full = tile_valid;  // every (query, key) pair of my 64 columns allowed?
+        if (p.causal) full = full && (U.k0 + 127 <= q0);
+        if (p.window >= 0) full = full && (q0 + 63 - U.k0 <= p.window) && (U.k0 + 127 - q0 <= p.window);
+        // (warp-uniform outcomes: the TMEM loads and stores below are warp-collective)
+        ok = mbar_wait(&q_full[s], (g / C::kQStages) & 1, abort_flag);  // LSE / D landed
+        ok = ok && mbar_wait(s_full, g & 1, abort_flag);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        if (lane == 0 && wl == 0) FA_TRACE_AT(w, g, 0);
+        tc_fence_after();
+        float pv[64];  // the fp32 weights P^T of my 64 columns
+        {
+          uint32_t sv[64];
+          tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 64; ++c) pv[c] = __uint_as_float(sv[c]);
-      }
-      if (full)
-        exp_cols64<true>(pv, nLv, sl2);
-      else
-        exp_cols64<false>(pv, nLv, sl2);
-      if (!full) {  // tiles on the diagonal / window edge only: one branch, not one per element
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int q = q0 + c;
-          bool keep = key_valid;
-          if (p.causal) keep = keep && key <= q;
-          if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
-          pv[c] = keep ? pv[c] : 0.f;
+          for (int c = 0; c < 64; ++c) pv[c] = __uint_as_float(sv[c]);
         }
-      }
-      {
-        uint32_t pk[32];  // my 64 P^T values, packed bf16: the A operand of dV += P^T dO
+        if (full)
+          exp_cols64<true>(pv, nLv, sl2);
+        else
+          exp_cols64<false>(pv, nLv, sl2);
+        if (!full) {  // tiles on the diagonal / window edge only: one branch, not one per element
 #pragma unroll
-        for (int u = 0; u < 32; ++u) pk[u] = pack_bf16x2(pv[2 * u], pv[2 * u + 1]);
-        tmem_st32(tS, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(p_full);
-      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 1);
+          for (int c = 0; c < 64; ++c) {
+            const int q = q0 + c;
+            bool keep = key_valid;
+            if (p.causal) keep = keep && key <= q;
+            if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
+            pv[c] = keep ? pv[c] : 0.f;
+          }
+        }
+        {
+          uint32_t pk[32];  // my 64 P^T values, packed bf16: the A operand of dV += P^T dO
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) pk[c2] = pack_bf16x2(pv[2 * c2], pv[2 * c2 + 1]);
+          tmem_st32(tS, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        if (lane == 0 && wl == 0) FA_TRACE_AT(w, g, 1);
 
-      ok = mbar_wait(dp_full, it & 1, abort_flag);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 2);
-      tc_fence_after();
+        ok = mbar_wait(dp_full, g & 1, abort_flag);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        if (lane == 0 && wl == 0) FA_TRACE_AT(w, g, 2);
+        tc_fence_after();
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t dv[32];
-        tmem_ld32(tDP + 32 * h, dv);
-        tmem_wait_ld();
-        uint32_t ds[16];
+        for (int h = 0; h < 2; ++h) {
+          uint32_t dv[32];
+          tmem_ld32(tDP + 32 * h, dv);
+          tmem_wait_ld();
+          uint32_t ds[16];
 #pragma unroll
-        for (int u2 = 0; u2 < 8; ++u2) {
-          const float4 d4 = reinterpret_cast<const float4*>(nDv)[8 * h + u2];
-          // dS = P (dP - D) on packed pairs, P kept in fp32 since the exponent phase
-          const int c = 32 * h + 4 * u2;
-          float a0, a1, a2, a3;
-          f2_split(fmul2(f2(pv[c], pv[c + 1]),
-                         fadd2(f2(__uint_as_float(dv[4 * u2]), __uint_as_float(dv[4 * u2 + 1])), f2(d4.x, d4.y))),
-                   a0, a1);
-          f2_split(fmul2(f2(pv[c + 2], pv[c + 3]),
-                         fadd2(f2(__uint_as_float(dv[4 * u2 + 2]), __uint_as_float(dv[4 * u2 + 3])), f2(d4.z, d4.w))),
-                   a2, a3);
-          ds[2 * u2] = pack_bf16x2(a0, a1);
-          ds[2 * u2 + 1] = pack_bf16x2(a2, a3);
+          for (int u2 = 0; u2 < 8; ++u2) {
+            const float4 d4 = reinterpret_cast<const float4*>(nDv)[8 * h + u2];
+            // dS = P (dP - D) on packed pairs, P kept in fp32 since the exponent phase
+            const int c = 32 * h + 4 * u2;
+            float a0, a1, a2, a3;
+            f2_split(fmul2(f2(pv[c], pv[c + 1]),
+                           fadd2(f2(__uint_as_float(dv[4 * u2]), __uint_as_float(dv[4 * u2 + 1])), f2(d4.x, d4.y))),
+                     a0, a1);
+            f2_split(fmul2(f2(pv[c + 2], pv[c + 3]), fadd2(f2(__uint_as_float(dv[4 * u2 + 2]),
+                                                              __uint_as_float(dv[4 * u2 + 3])),
+                                                           f2(d4.z, d4.w))),
+                     a2, a3);
+            ds[2 * u2] = pack_bf16x2(a0, a1);
+            ds[2 * u2 + 1] = pack_bf16x2(a2, a3);
+          }
+          // dS^T (packed) over dP^T columns this thread has already read; dS into
+          // shared memory as rows = keys, columns = queries (MN-major A of dQ).
+          tmem_st16(tDP + 16 * h, ds);
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            const int unit16 = h * 4 + u4;  // 16-byte unit within my 128-byte row chunk
+            *reinterpret_cast<uint4*>(sDS + ds_chunk * 16384 + r * 128 + ((unit16 ^ (r & 7)) << 4)) =
+                make_uint4(ds[4 * u4], ds[4 * u4 + 1], ds[4 * u4 + 2], ds[4 * u4 + 3]);
+          }
         }
-        // dS^T (packed) over dP^T columns this thread has already read; dS into
-        // shared memory as rows = keys, columns = queries (MN-major A of dQ).
-        tmem_st16(tDP + 16 * h, ds);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = h * 4 + u;  // 16-byte unit within my 128-byte row chunk
-          *reinterpret_cast<uint4*>(sDS + ds_chunk * 16384 + r * 128 + ((unit ^ (r & 7)) << 4)) =
-              make_uint4(ds[4 * u], ds[4 * u + 1], ds[4 * u + 2], ds[4 * u + 3]);
-        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(ds_full);
+        if (lane == 0 && wl == 0) FA_TRACE_AT(w, g, 3);
       }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(ds_full);
-      if (lane == 0 && wl == 0) FA_TRACE_AT(w, it, 3);
+      git += U.total;
     }
   } else {
-    // ------------------------------------------------------------ dQ drain, then dK/dV epilogue
-    regs_inc<160>();
+    // ------------------------------------------------------------ dQ drain and the dK/dV epilogue
+    regs_inc<kBwdRegsDrain>();
     const int wl = warp & 3;
     const int r = wl * 32 + lane;  // query row of the dQ tile (drain), key row (epilogue)
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
     constexpr int kBarDrain = 1, kBarDrainAnd = 2;  // named barriers of the 128 drain threads
     bool ok = true;
     int nchunk = 0;  // chunks handed to the TMA unit so far
-    QCursor cur = first();
-    for (int it = 0; it < total; ++it, cur = advance(cur)) {
-      ok = mbar_wait(dq_full, it & 1, abort_flag);
-      // all 128 threads take the same branch: the named barriers below need every one of them
-      if (!(ok = named_bar_and(kBarDrainAnd, 128, ok))) break;
-      if (r == 0) FA_TRACE_AT(4, it, 0);
-      tc_fence_after();
-      uint32_t v[D];
+    int git = 0;
+    for (int u = 0; ok && u < nunits; ++u) {
+      const Unit U = unit(u);
+      QCursor cur = first(U);
+      for (int it = 0; it < U.total; ++it, cur = advance(U, cur)) {
+        const int g = git + it;
+        ok = mbar_wait(dq_full, g & 1, abort_flag);
+        // all 128 threads take the same branch: the named barriers below need every one of them
+        if (!(ok = named_bar_and(kBarDrainAnd, 128, ok))) break;
+        if (r == 0) FA_TRACE_AT(4, g, 0);
+        tc_fence_after();
+        uint32_t v[D];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c)
-        tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(dq_empty);  // TMEM tile free before the reductions are staged
-      if (r == 0) FA_TRACE_AT(4, it, 1);
-      const size_t bh = static_cast<size_t>(bh0 + cur.hq);
+        for (int c = 0; c < D / 32; ++c)
+          tmem_ld32(tmem + lane_off + C::kColDQ + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(dq_empty);  // TMEM tile free before the reductions are staged
+        if (r == 0) FA_TRACE_AT(4, g, 1);
+        const size_t bh = static_cast<size_t>(bh0 + cur.hq);
 #pragma unroll
-      for (int c = 0; c < C::kDqChunks; ++c, ++nchunk) {
-        uint8_t* buf = sDQ + (nchunk % C::kDqStages) * C::kDqChunkBytes;
-        // the buffer's previous chunk has been read by the TMA unit
-        if (r == 0 && nchunk >= C::kDqStages) bulk_wait_read<C::kDqStages - 1>();
-        named_bar_sync(kBarDrain, 128);
+        for (int c = 0; c < C::kDqChunks; ++c, ++nchunk) {
+          uint8_t* buf = sDQ + (nchunk % C::kDqStages) * C::kDqChunkBytes;
+          // the buffer's previous chunk has been read by the TMA unit
+          if (r == 0 && nchunk >= C::kDqStages) bulk_wait_read<C::kDqStages - 1>();
+          named_bar_sync(kBarDrain, 128);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          *reinterpret_cast<uint4*>(buf + r * 128 + ((u ^ (r & 7)) << 4)) =
-              make_uint4(v[c * 32 + 4 * u], v[c * 32 + 4 * u + 1], v[c * 32 + 4 * u + 2], v[c * 32 + 4 * u + 3]);
-        fence_proxy_async_smem();
-        named_bar_sync(kBarDrain, 128);
-        if (r == 0) {
-          bulk_reduce_add_f32(p.dqacc + dqacc_chunk<D>(bh, p.ntiles, cur.i, c), buf, C::kDqChunkBytes);
-          bulk_commit();
+          for (int u8 = 0; u8 < 8; ++u8)
+            *reinterpret_cast<uint4*>(buf + r * 128 + ((u8 ^ (r & 7)) << 4)) =
+                make_uint4(v[c * 32 + 4 * u8], v[c * 32 + 4 * u8 + 1], v[c * 32 + 4 * u8 + 2],
+                           v[c * 32 + 4 * u8 + 3]);
+          fence_proxy_async_smem();
+          named_bar_sync(kBarDrain, 128);
+          if (r == 0) {
+            bulk_reduce_add_f32(p.dqacc + dqacc_chunk<D>(bh, p.ntiles, cur.i, c), buf, C::kDqChunkBytes);
+            bulk_commit();
+          }
         }
+        if (r == 0) FA_TRACE_AT(4, g, 2);
       }
-      if (r == 0) FA_TRACE_AT(4, it, 2);
-    }
-    if (r == 0) bulk_wait0();  // every reduction complete before the CTA exits
-    if (ok) ok = mbar_wait(kv_done, 0, abort_flag);
-    ok = named_bar_and(kBarDrainAnd, 128, ok);  // the TMEM loads below are warp-collective
-    if (ok) {
+      if (!ok) break;
+      git += U.total;
+      // ---- epilogue of the unit: dV and dK (x scale) to bf16, through the staging buffers
+      ok = named_bar_and(kBarDrainAnd, 128, mbar_wait(kv_done, u & 1, abort_flag));
+      if (!ok) break;
       tc_fence_after();
-      // K and V tiles are no longer read: stage dV over V and dK over K.
+      if (r == 0) bulk_wait_read0();  // staging buffers no longer read by earlier reductions
+      named_bar_sync(kBarDrain, 128);
+      uint8_t* sDV = sDQ;                                  // bf16 128 x D tile in the TMA layout
+      uint8_t* sDK = sDQ + (D == 128 ? 0 : C::kTileBytes);  // after dV's store has read it (D = 128)
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
-        uint32_t v[32];
-        if (total > 0) {
-          tmem_ld32(tmem + lane_off + C::kColDV + c, v);
+        uint32_t t[32];
+        if (U.total > 0) {
+          tmem_ld32(tmem + lane_off + C::kColDV + c, t);
           tmem_wait_ld();
-        } else {  // no query block reaches this key tile (block mask): dV = dK = 0
+        } else {  // no query block reaches this key tile: dV = dK = 0
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = 0u;
+          for (int i = 0; i < 32; ++i) t[i] = 0u;
         }
-        stage_row32_bf16(sV, r, c, v, 1.f);
-        if (total > 0) {
-          tmem_ld32(tmem + lane_off + C::kColDK + c, v);
-          tmem_wait_ld();
-        }
-        stage_row32_bf16(sK, r, c, v, p.scale);
+        stage_row32_bf16(sDV, r, c, t, 1.f);
       }
-      fence_proxy_async_smem();
-    }
-    mbar_arrive(epi_bar);
-    if (ok && r == 0 && mbar_wait(epi_bar, 0, abort_flag)) {
-      for (int c = 0; c < C::kChunks; ++c) {
-        if constexpr (kStrided) {
-          tma_store_tile(&tmdV, p.map4 & kBMapDV, sV + c * 16384, c * 64, k0, bkv, kh, b);
-          tma_store_tile(&tmdK, p.map4 & kBMapDK, sK + c * 16384, c * 64, k0, bkv, kh, b);
+      uint32_t v[D];  // dK row, held while dV's store reads the staging buffers
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        if (U.total > 0) {
+          tmem_ld32(tmem + lane_off + C::kColDK + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
         } else {
-          tma_store_3d(&tmdV, sV + c * 16384, c * 64, k0, bkv);
-          tma_store_3d(&tmdK, sK + c * 16384, c * 64, k0, bkv);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[c * 32 + i] = 0u;
         }
       }
-      bulk_commit();
-      bulk_wait0();
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(acc_empty);  // the next unit's products may overwrite dV and dK
+      fence_proxy_async_smem();
+      named_bar_sync(kBarDrain, 128);
+      if (r == 0) {
+        for (int c = 0; c < C::kChunks; ++c) {
+          if constexpr (kStrided)
+            tma_store_tile(&tmdV, p.map4 & kBMapDV, sDV + c * 16384, c * 64, U.k0, bkv, kh, b);
+          else
+            tma_store_3d(&tmdV, sDV + c * 16384, c * 64, U.k0, bkv);
+        }
+        bulk_commit();
+        if (D == 128) bulk_wait_read0();  // dK reuses the buffers dV's store reads
+      }
+      named_bar_sync(kBarDrain, 128);
+#pragma unroll
+      for (int c = 0; c < D; c += 32)
+        stage_row32_bf16(sDK, r, c, *reinterpret_cast<const uint32_t(*)[32]>(&v[c]), p.scale);
+      fence_proxy_async_smem();
+      named_bar_sync(kBarDrain, 128);
+      if (r == 0) {
+        for (int c = 0; c < C::kChunks; ++c) {
+          if constexpr (kStrided)
+            tma_store_tile(&tmdK, p.map4 & kBMapDK, sDK + c * 16384, c * 64, U.k0, bkv, kh, b);
+          else
+            tma_store_3d(&tmdK, sDK + c * 16384, c * 64, U.k0, bkv);
+        }
+        bulk_commit();
+        bulk_wait_read0();  // the next unit's dQ chunks reuse the staging buffers
+      }
+      named_bar_sync(kBarDrain, 128);
     }
+    if (r == 0) bulk_wait0();  // every reduction and store complete before the CTA exits
   }
   tc_fence_before();
   __syncthreads();

@@ -402,6 +402,8 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   p.causal = causal ? 1 : 0;
   p.window = window;
   p.ntiles = p.Np / 128;
+  p.slots = (p.ntiles + 1) / 2;
+  p.pairs = (causal && window < 0) ? 1 : 0;
   p.bmask = bmask;
   p.bmask_hs = bmask_hs;
   p.seqlens = seqlens;
@@ -425,7 +427,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
     return FA_ERR_CUDA;
   const size_t rows = static_cast<size_t>(B) * H * p.Np;
   const unsigned pre_grid = static_cast<unsigned>((rows + 8 * fa::kPreRowsPerWarp - 1) / (8 * fa::kPreRowsPerWarp));
-  const unsigned grid = static_cast<unsigned>(p.ntiles) * B * Hkv;
+  const unsigned grid = static_cast<unsigned>(p.slots) * B * Hkv;
   const unsigned dq_grid = static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32));
   if (L) {
     if (bmask) return FA_ERR_UNSUPPORTED;
