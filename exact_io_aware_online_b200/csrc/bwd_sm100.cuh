@@ -74,8 +74,9 @@ struct BwdParams {
   int causal, window;
   int ntiles;  // Np / 128
   int group;   // kv heads per rasterisation group (kept L2-resident together)
-  int slots;   // CTAs per kv head: ceil(ntiles / 2), each running up to two key tiles
-  int pairs;   // 1: a CTA runs key tiles j and ntiles - 1 - j (causal); 0: tiles 2j and 2j + 1
+  int slots;   // CTAs per kv head
+  int pairs;   // 1 (causal): ceil(ntiles / 2) CTAs, each running key tiles j and ntiles - 1 - j;
+               // 0: ntiles CTAs, one key tile each
   // block-sparse mode (non-null bmask): 0/1 per 128 x 128 block, [query block]
   // [key block] per query head, bmask_hs elements apart (0: shared by all heads)
   const uint8_t* bmask;
@@ -121,6 +122,9 @@ struct BwdCfg {
   static constexpr bool kAliasDq = (D == 128);
   static constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
   static constexpr uint32_t kColDQ = kAliasDq ? 128 : 256 + 2 * D;
+  // Exponentials all on the special-function unit: the polynomial on the FMA
+  // pipe costs more issue slots than it frees here (measured at D = 64 and 128).
+  static constexpr bool kPolyExp = false;
 };
 static_assert(BwdCfg<128>::kSmemBytes <= 232448, "backward shared memory over the per-CTA limit");
 // Per-thread register budgets after setmaxnreg (compute, compute, drain, MMA +
@@ -278,12 +282,12 @@ __device__ __forceinline__ void exp_cols64(float (&x)[64], const float* nLv, flo
 }
 
 // ---------------------------------------------------------------- main kernel
-// Work units are (kv head, 128-key tile) pairs; each CTA runs up to two units
-// of one kv head back to back, its pipelines running on from the first unit
-// into the second.  Under a causal mask the two are key tiles j and
-// ntiles - 1 - j, whose query-tile counts add up to the same total for every
-// CTA, so the grid has no long and short CTAs; otherwise they are adjacent
-// tiles (which share most of their query tiles in a window band).
+// Work units are (kv head, 128-key tile) pairs.  Under a causal mask each CTA
+// runs two units of one kv head back to back, key tiles j and ntiles - 1 - j,
+// whose query-tile counts add up to the same total for every CTA (so the grid
+// has no long and short CTAs), its pipelines running on from the first unit
+// into the second.  Otherwise every unit has about the same work and each CTA
+// runs one.
 constexpr int kBwdMaxUnits = 2;
 
 template <int D, bool kMask, bool kStrided = false>
@@ -339,7 +343,7 @@ __global__ void __launch_bounds__(512, 1)
   const int b = bkv / p.Hkv, kh = bkv % p.Hkv;
   const int Lb = valid_rows(p, b);
   const int bh0 = b * p.H + kh * p.g;  // first query head of the GQA group
-  const int nunits = p.pairs ? (p.ntiles - 1 - slot != slot ? 2 : 1) : (2 * slot + 1 < p.ntiles ? 2 : 1);
+  const int nunits = p.pairs ? (p.ntiles - 1 - slot != slot ? 2 : 1) : 1;
   // One unit: key tile j, its query-tile range [ilo, ihi] and the number of
   // (query head, query tile) work items.  Work items are walked in increasing
   // order, skipping blocks a block-sparse mask switches off; every role walks
@@ -370,7 +374,7 @@ __global__ void __launch_bounds__(512, 1)
   };
   auto unit = [&](int u) {
     Unit U;
-    U.j = p.pairs ? (u == 0 ? slot : p.ntiles - 1 - slot) : 2 * slot + u;
+    U.j = p.pairs ? (u == 0 ? slot : p.ntiles - 1 - slot) : slot;
     U.k0 = U.j * 128;
     U.ilo = 0;
     U.ihi = (max(Lb, 1) - 1) / 128;  // query tiles holding valid rows
@@ -670,19 +674,23 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int c = 0; c < 64; ++c) pv[c] = __uint_as_float(sv[c]);
         }
-        if (full)
+        if (full && C::kPolyExp)
           exp_cols64<true>(pv, nLv, sl2);
         else
           exp_cols64<false>(pv, nLv, sl2);
-        if (!full) {  // tiles on the diagonal / window edge only: one branch, not one per element
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int q = q0 + c;
-            bool keep = key_valid;
-            if (p.causal) keep = keep && key <= q;
-            if (p.window >= 0) keep = keep && abs(q - key) <= p.window;
-            pv[c] = keep ? pv[c] : 0.f;
+        if (!full) {
+          // Tiles on the diagonal / window edge only: my key row may see query
+          // columns [c_lo, c_hi] of my 64; one unsigned compare per element.
+          int c_lo = 0, c_hi = key_valid ? 63 : -1;
+          if (p.causal) c_lo = max(c_lo, key - q0);
+          if (p.window >= 0) {
+            c_lo = max(c_lo, key - p.window - q0);
+            c_hi = min(c_hi, key + p.window - q0);
           }
+          if (c_hi < c_lo) c_lo = 64, c_hi = 64;  // nothing allowed: (c - 64) wraps above the span
+          const uint32_t span = static_cast<uint32_t>(c_hi - c_lo);
+#pragma unroll
+          for (int c = 0; c < 64; ++c) pv[c] = static_cast<uint32_t>(c - c_lo) <= span ? pv[c] : 0.f;
         }
         {
           uint32_t pk[32];  // my 64 P^T values, packed bf16: the A operand of dV += P^T dO
@@ -853,7 +861,9 @@ __global__ void __launch_bounds__(512, 1)
       }
       named_bar_sync(kBarDrain, 128);
     }
-    if (r == 0) bulk_wait0();  // every reduction and store complete before the CTA exits
+    // Shared memory must outlive the copies that read it; the global side of the
+    // reductions and stores completes with the grid.
+    if (r == 0) bulk_wait_read0();
   }
   tc_fence_before();
   __syncthreads();

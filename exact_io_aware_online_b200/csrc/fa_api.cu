@@ -402,8 +402,8 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   p.causal = causal ? 1 : 0;
   p.window = window;
   p.ntiles = p.Np / 128;
-  p.slots = (p.ntiles + 1) / 2;
   p.pairs = (causal && window < 0) ? 1 : 0;
+  p.slots = p.pairs ? (p.ntiles + 1) / 2 : p.ntiles;
   p.bmask = bmask;
   p.bmask_hs = bmask_hs;
   p.seqlens = seqlens;

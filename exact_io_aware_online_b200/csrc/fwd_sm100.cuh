@@ -110,6 +110,10 @@ struct FwdCfg {
   static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + 8 * kNumBars + 16;
   static constexpr int kThreads = 384;
   static constexpr uint32_t kTmemCols = 512;
+  // A quarter of the exponentials on the FMA pipe (exp2_poly2) pays at D = 64,
+  // where the special-function unit does twice the work per tensor-core cycle;
+  // at D = 128 the extra instructions cost more than they save (measured).
+  static constexpr bool kPolyExp = (D == 64);
 };
 
 constexpr float kTau = 8.0f;  // lazy-rescale threshold, log2 units (factor 256)
@@ -263,6 +267,14 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) {
+    FA_TRACE_AT(6, 0, 0);
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    FA_TRACE_CTA(0, smid);
+    FA_TRACE_CTA(1, nkv);
+    FA_TRACE_CTA(2, globaltimer_ns());
+  }
 
   if (warp >= 8) {
     regs_dec<72>();
@@ -406,6 +418,7 @@ __global__ void __launch_bounds__(384, 1)
       // (warp-uniform outcome: the TMEM loads and stores below are warp-collective)
       ok = mbar_wait(&s_full[t], jj & 1, abort_flag);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      if (lane == 0 && wl == 0) FA_TRACE_AT(t, jj, 0);
       tc_fence_after();
       if (kMask && block_off) {  // every weight of the tile is zero: store P = 0 and move on
         uint32_t z[16];
@@ -429,14 +442,18 @@ __global__ void __launch_bounds__(384, 1)
       if (p.causal) full = full && (kv0 + 127 <= tpmin);
       if (p.window >= 0) full = full && (tpmax - kv0 <= p.window) && (kv0 + 127 - tpmin <= p.window);
       if (!full) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const int key = kv0 + c;
-          bool keep = key < Lk && !block_off;
-          if (p.causal) keep = keep && key <= qpos;
-          if (p.window >= 0) keep = keep && abs(qpos - key) <= p.window;
-          if (!keep) s[c] = -INFINITY;
+        // Tiles on the diagonal / window edge / sequence end only: my row may
+        // see key columns [c_lo, c_hi] of the tile; one unsigned compare per element.
+        int c_lo = 0, c_hi = block_off ? -1 : min(127, Lk - 1 - kv0);
+        if (p.causal) c_hi = min(c_hi, qpos - kv0);
+        if (p.window >= 0) {
+          c_lo = max(c_lo, qpos - p.window - kv0);
+          c_hi = min(c_hi, qpos + p.window - kv0);
         }
+        if (c_hi < c_lo) c_lo = 128, c_hi = 128;  // nothing allowed: (c - 128) wraps above the span
+        const uint32_t span = static_cast<uint32_t>(c_hi - c_lo);
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = static_cast<uint32_t>(c - c_lo) <= span ? s[c] : -INFINITY;
       }
       float mx8[8];  // eight independent partial maxima (short dependency chains)
 #pragma unroll
@@ -472,13 +489,14 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_st();
       }
       const float ms = (m_used == -INFINITY) ? 0.f : m_used;
-      if (full)
+      if (full && C::kPolyExp)
         exp_row_to_tmem<true>(s, sl2, ms, tS, l, lb);
       else
         exp_row_to_tmem<false>(s, sl2, ms, tS, l, lb);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[t]);
+      if (lane == 0 && wl == 0) FA_TRACE_AT(t, jj, 1);
     }
     if (kSplit) {
       // ------------------------------------------------ partial results
@@ -558,6 +576,10 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
+  }
+  if (threadIdx.x == 0) {
+    FA_TRACE_AT(6, 0, 1);
+    FA_TRACE_CTA(3, globaltimer_ns());
   }
 }
 

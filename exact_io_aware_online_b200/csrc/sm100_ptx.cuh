@@ -183,20 +183,6 @@ __device__ __forceinline__ void tma_store_tile(const CUtensorMap* map, bool four
   else
     tma_store_3d(map, src, c, row, idx);
 }
-// Hint: bring a tile into L2 ahead of its load (no completion to wait for).
-__device__ __forceinline__ void tma_prefetch_tile(const CUtensorMap* map, bool four, int c, int row, int idx, int h,
-                                                  int b) {
-  if (four)
-    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c), "r"(row), "r"(h), "r"(b)
-                 : "memory");
-  else
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c), "r"(row), "r"(idx)
-                 : "memory");
-}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Waits until at most N committed bulk groups of this thread still read shared memory.
