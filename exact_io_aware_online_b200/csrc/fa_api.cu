@@ -73,8 +73,8 @@ EncodeTiledFn get_encode() {
 // (d, N, heads, B); *four reports which.  Rows past N are zero-filled on load
 // and clipped on store, so a tile never reaches another head's or batch
 // entry's rows whatever the strides.
-bool make_tile_map(CUtensorMap* m, const void* ptr, int B, int heads, int N, int d, const fa::Strides& s,
-                   bool* four) {
+bool encode_tile_map(CUtensorMap* m, const void* ptr, int B, int heads, int N, int d, const fa::Strides& s,
+                     bool* four) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   *four = !(B == 1 || s.b == static_cast<long long>(heads) * s.h);
@@ -89,6 +89,49 @@ bool make_tile_map(CUtensorMap* m, const void* ptr, int B, int heads, int N, int
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Encoded maps are cached by everything they encode (address, sizes, strides):
+// a hit is exactly the map a fresh encode would give, so the cache needs no
+// invalidation when buffers are freed and reused.  A small ring, shared by all
+// threads under a mutex.
+struct TileMapKey {
+  const void* ptr;
+  int B, heads, N, d;
+  long long sb, sh, sn;
+  bool operator==(const TileMapKey& o) const {
+    return ptr == o.ptr && B == o.B && heads == o.heads && N == o.N && d == o.d && sb == o.sb && sh == o.sh &&
+           sn == o.sn;
+  }
+};
+struct TileMapEntry {
+  TileMapKey key;
+  CUtensorMap map;
+  bool four;
+  bool used;
+};
+constexpr int kTileMapCache = 64;
+
+bool make_tile_map(CUtensorMap* m, const void* ptr, int B, int heads, int N, int d, const fa::Strides& s,
+                   bool* four) {
+  static std::mutex mu;
+  static TileMapEntry cache[kTileMapCache];
+  static int next = 0;
+  const TileMapKey key{ptr, B, heads, N, d, s.b, s.h, s.n};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const TileMapEntry& e : cache)
+      if (e.used && e.key == key) {
+        *m = e.map;
+        *four = e.four;
+        return true;
+      }
+  }
+  if (!encode_tile_map(m, ptr, B, heads, N, d, s, four)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  cache[next] = TileMapEntry{key, *m, *four, true};
+  next = (next + 1) % kTileMapCache;
+  return true;
 }
 
 // Element strides of every tensor argument of one call.
@@ -144,9 +187,26 @@ fa_status check_strides(const fa::Strides& s, int B, int heads, int N, int d, in
   return FA_OK;
 }
 
+// Raises a kernel's dynamic shared-memory limit, once per (kernel, device):
+// the raised limits are remembered by kernel address and device.
 template <typename K>
 bool set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+  struct Done {
+    const void* fn;
+    int dev, bytes;
+  };
+  static std::mutex mu;
+  static Done done[256];
+  static int ndone = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < ndone; ++i)
+    if (done[i].fn == fn && done[i].dev == dev && done[i].bytes == bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (ndone < 256) done[ndone++] = Done{fn, dev, bytes};
+  return true;
 }
 
 // Launches one kernel and reports that launch's own outcome (an error left
