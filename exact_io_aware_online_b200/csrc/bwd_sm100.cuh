@@ -11,12 +11,12 @@
 // Three kernels run on one stream:
 //   bwd_pre_kernel   -D_i, -LSE_i * log2(e) (-inf on padding rows) and a
 //                    zeroed fp32 dQ accumulator, all in the caller's workspace;
-//   bwd_sm100_kernel one CTA per (batch, kv head, pair of 128-key tiles): for
-//                    each tile j, K_j and V_j stay in shared memory while the
-//                    CTA walks every query tile (of every query head of the
-//                    GQA group) that can see them; dK_j and dV_j accumulate in
-//                    TMEM and are written once, dQ partial tiles are added
-//                    into the accumulator;
+//   bwd_sm100_kernel persistent: each CTA runs a list of jobs, one 128-key tile
+//                    of one kv head each: K_j and V_j stay in shared memory
+//                    while the CTA walks every query tile (of every query head
+//                    of the GQA group) that can see them; dK_j and dV_j
+//                    accumulate in TMEM and are written once, dQ partial tiles
+//                    are added into the accumulator;
 //   bwd_dq_kernel    dQ = bf16(scale * accumulator).
 //
 // Main-kernel roles (512 threads, four warpgroups):
@@ -107,16 +107,19 @@ struct BwdCfg {
   static constexpr int kChunks = D / 64;                 // 64-column chunks of a bf16 tile
   static constexpr int kQStages = (D == 128) ? 2 : 3;    // (Q, LSE, D) tile sets in flight
   static constexpr int kDoStages = (D == 128) ? 1 : 2;   // dO tiles in flight
+  // K/V buffers: with two, the next job's K and V load while the current job
+  // runs (no room for a second pair at D = 128).
+  static constexpr int kKvBufs = (D == 128) ? 1 : 2;
   static constexpr int kDsBytes = 128 * 128 * 2;
   static constexpr int kVecBytes = 2 * 128 * 4;          // -LSE*log2(e) and -D of one query tile
   static constexpr int kDqChunkBytes = 128 * 32 * 4;     // 32 fp32 columns of a 128-row dQ tile
   static constexpr int kDqChunks = D / 32;               // chunks per dQ tile
   static constexpr int kDqStages = 2;                    // staging buffers of the dQ reduction
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 * kDoStages + 11;
+  static constexpr int kNumBars = 2 * kKvBufs + 2 * kQStages + 2 * kDoStages + 9;
   // The dynamic shared window starts 1024-byte aligned (checked at run time),
-  // so no alignment slack is reserved: at D = 128 this is 231,584 of the
-  // 232,448 bytes a CTA may use.
-  static constexpr int kSmemBytes = 2 * kTileBytes + kQStages * kTileBytes + kDoStages * kTileBytes + kDsBytes +
+  // so no alignment slack is reserved: at D = 128 this is 231,576 of the
+  // 232,448 bytes a CTA may use (216,264 at D = 64).
+  static constexpr int kSmemBytes = 2 * kKvBufs * kTileBytes + kQStages * kTileBytes + kDoStages * kTileBytes + kDsBytes +
                                     kDqStages * kDqChunkBytes + kQStages * kVecBytes + 8 * kNumBars + 16;
   static constexpr int kThreads = 512;
   static constexpr bool kAliasDq = (D == 128);
@@ -126,7 +129,8 @@ struct BwdCfg {
   // pipe costs more issue slots than it frees here (measured at D = 64 and 128).
   static constexpr bool kPolyExp = false;
 };
-static_assert(BwdCfg<128>::kSmemBytes <= 232448, "backward shared memory over the per-CTA limit");
+static_assert(BwdCfg<128>::kSmemBytes <= 232448 && BwdCfg<64>::kSmemBytes <= 232448,
+              "backward shared memory over the per-CTA limit");
 // Per-thread register budgets after setmaxnreg (compute, compute, drain, MMA +
 // producers): an increase waits until decreases have freed the registers, so
 // the four must add up to the 4 x 128 the 512-thread launch provides.
@@ -282,13 +286,14 @@ __device__ __forceinline__ void exp_cols64(float (&x)[64], const float* nLv, flo
 }
 
 // ---------------------------------------------------------------- main kernel
-// Work units are (kv head, 128-key tile) pairs.  Under a causal mask each CTA
-// runs two units of one kv head back to back, key tiles j and ntiles - 1 - j,
-// whose query-tile counts add up to the same total for every CTA (so the grid
-// has no long and short CTAs), its pipelines running on from the first unit
-// into the second.  Otherwise every unit has about the same work and each CTA
-// runs one.
-constexpr int kBwdMaxUnits = 2;
+// Work: slots numbered over (rasterisation group, slot, kv head), each holding
+// one 128-key tile of one kv head, or under a causal mask two, key tiles j and
+// ntiles - 1 - j, whose query-tile counts add up to the same total for every
+// slot.  CTA c runs slots c, c + gridDim.x, c + 2 gridDim.x, ... (the grid is
+// at most one CTA per SM), one job (key tile) after another, with every
+// pipeline running on from one job into the next: the next job's Q and dO
+// tiles load while the current one finishes, and its first products start
+// while the drain warpgroup writes the current job's dK and dV.
 
 template <int D, bool kMask, bool kStrided = false>
 __global__ void __launch_bounds__(512, 1)
@@ -302,16 +307,16 @@ __global__ void __launch_bounds__(512, 1)
     if (threadIdx.x == 0) atomicOr(&g_status, kStatusMisaligned);
     return;
   }
-  uint8_t* sK = smem_raw;
-  uint8_t* sV = smem_raw + C::kTileBytes;
-  uint8_t* sQ = smem_raw + 2 * C::kTileBytes;              // Q stage s at s * kTileBytes
+  uint8_t* sKV = smem_raw;                                 // K/V buffer kb: K at 2 kb kTileBytes, V after it
+  uint8_t* sQ = smem_raw + 2 * C::kKvBufs * C::kTileBytes;  // Q stage s at s * kTileBytes
   uint8_t* sDO = sQ + C::kQStages * C::kTileBytes;        // dO stage s at s * kTileBytes
   uint8_t* sDS = sDO + C::kDoStages * C::kTileBytes;
   uint8_t* sDQ = sDS + C::kDsBytes;  // dQ staging buffers, kDqChunkBytes each; dK/dV epilogue staging
   uint8_t* sVec = sDQ + C::kDqStages * C::kDqChunkBytes;  // Q stage s: -LSE*log2(e) [128] then -D [128]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sVec + C::kQStages * C::kVecBytes);
-  uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;
+  uint64_t* kv_full = bars;                 // per K/V buffer
+  uint64_t* kv_empty = bars + C::kKvBufs;   // per K/V buffer: a job's products no longer read it
+  uint64_t* q_full = bars + 2 * C::kKvBufs;
   uint64_t* q_empty = q_full + C::kQStages;
   uint64_t* do_full = q_empty + C::kQStages;
   uint64_t* do_empty = do_full + C::kDoStages;
@@ -321,42 +326,52 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* ds_full = s_full + 3;
   uint64_t* dq_full = s_full + 4;
   uint64_t* dq_empty = s_full + 5;
-  uint64_t* kv_done = s_full + 6;    // a unit's dV and dK are complete in TMEM
-  uint64_t* kv_empty = s_full + 7;   // a unit's products no longer read K and V
-  uint64_t* acc_empty = s_full + 8;  // a unit's dV and dK have been read out of TMEM
-  uint64_t* mma_idle = s_full + 9;   // every product the MMA thread issued has completed
+  uint64_t* kv_done = s_full + 6;    // a job's dV and dK are complete in TMEM
+  uint64_t* acc_empty = s_full + 7;  // a job's dV and dK have been read out of TMEM
+  uint64_t* mma_idle = s_full + 8;   // every product the MMA thread issued has completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- this CTA's kv head and slot.  Groups of p.group kv heads run together
-  // (their Q, dO, K, V and dQ accumulator stay in L2).
+  // ---- this CTA's jobs.  Slots are numbered group-major: groups of p.group
+  // kv heads run together (their Q, dO, K, V and dQ accumulator stay in L2).
   const int BHkv = p.B * p.Hkv;
-  const int per_group = p.group * p.slots;
-  const int grp = static_cast<int>(blockIdx.x) / per_group;
-  const int g0 = grp * p.group;
-  const int gsz = min(p.group, BHkv - g0);
-  const int rem = static_cast<int>(blockIdx.x) - grp * per_group;
-  const int slot = rem / gsz;
-  const int bkv = g0 + rem % gsz;
-  const int b = bkv / p.Hkv, kh = bkv % p.Hkv;
-  const int Lb = valid_rows(p, b);
-  const int bh0 = b * p.H + kh * p.g;  // first query head of the GQA group
-  const int nunits = p.pairs ? (p.ntiles - 1 - slot != slot ? 2 : 1) : 1;
-  // One unit: key tile j, its query-tile range [ilo, ihi] and the number of
-  // (query head, query tile) work items.  Work items are walked in increasing
-  // order, skipping blocks a block-sparse mask switches off; every role walks
-  // them with its own cursor, so all roles see the same sequence.
-  // (kMask: the block-sparse variant; the dense kernels compile no mask test.)
+  const int nslots = p.slots * BHkv;
+  struct Job {
+    int gs, sub;  // global slot, key tile within the slot
+  };
+  auto slot_of = [&](int gs, int& slot, int& bkv) {
+    const int per_group = p.group * p.slots;
+    const int grp = gs / per_group;
+    const int g0 = grp * p.group;
+    const int gsz = min(p.group, BHkv - g0);
+    const int rem = gs - grp * per_group;
+    slot = rem / gsz;
+    bkv = g0 + rem % gsz;
+  };
+  auto job_next = [&](Job J) {
+    int slot, bkv;
+    slot_of(J.gs, slot, bkv);
+    if (J.sub == 0 && p.pairs && p.ntiles - 1 - slot != slot) return Job{J.gs, 1};
+    return Job{J.gs + static_cast<int>(gridDim.x), 0};
+  };
+  const Job job0{static_cast<int>(blockIdx.x), 0};
+  // One job: key tile j of kv head bkv, its query-tile range [ilo, ihi] and the
+  // number of (query head, query tile) work items.  Work items are walked in
+  // increasing order, skipping blocks a block-sparse mask switches off; every
+  // role walks the same jobs and items with its own cursors, so all roles see
+  // the same sequence.  (kMask: the block-sparse variant; the dense kernels
+  // compile no mask test.)
   struct Unit {
     int j, k0, ilo, ihi, total;
+    int bkv, b, kh, bh0, Lb;  // kv head, batch entry, kv head in it, first query head, valid rows
   };
   struct QCursor {
     int hq, i;
   };
   auto active = [&](const Unit& U, int hq, int i) {
-    return !kMask || p.bmask[(bh0 + hq) * p.bmask_hs + static_cast<long long>(i) * p.ntiles + U.j] != 0;
+    return !kMask || p.bmask[(U.bh0 + hq) * p.bmask_hs + static_cast<long long>(i) * p.ntiles + U.j] != 0;
   };
   auto advance = [&](const Unit& U, QCursor c) {  // next active item strictly after c
     do {
@@ -372,18 +387,24 @@ __global__ void __launch_bounds__(512, 1)
     if (kMask && !active(U, 0, U.ilo)) c = advance(U, c);
     return c;
   };
-  auto unit = [&](int u) {
+  auto unit = [&](Job J) {
     Unit U;
-    U.j = p.pairs ? (u == 0 ? slot : p.ntiles - 1 - slot) : slot;
+    int slot;
+    slot_of(J.gs, slot, U.bkv);
+    U.b = U.bkv / p.Hkv;
+    U.kh = U.bkv % p.Hkv;
+    U.Lb = valid_rows(p, U.b);
+    U.bh0 = U.b * p.H + U.kh * p.g;
+    U.j = p.pairs ? (J.sub == 0 ? slot : p.ntiles - 1 - slot) : slot;
     U.k0 = U.j * 128;
     U.ilo = 0;
-    U.ihi = (max(Lb, 1) - 1) / 128;  // query tiles holding valid rows
+    U.ihi = (max(U.Lb, 1) - 1) / 128;  // query tiles holding valid rows
     if (p.causal) U.ilo = U.j;
     if (p.window >= 0) {
       U.ilo = max(U.ilo, max(0, U.k0 - p.window) / 128);
       U.ihi = min(U.ihi, (U.k0 + 127 + p.window) / 128);
     }
-    const bool no_work = U.ilo > U.ihi || U.k0 >= Lb;  // nothing reaches this key tile
+    const bool no_work = U.ilo > U.ihi || U.k0 >= U.Lb;  // nothing reaches this key tile
     U.total = no_work ? 0 : (U.ihi - U.ilo + 1) * p.g;
     if (kMask && !no_work) {
       U.total = 0;
@@ -393,7 +414,10 @@ __global__ void __launch_bounds__(512, 1)
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(kv_full, 1);
+    for (int i = 0; i < C::kKvBufs; ++i) {
+      mbar_init(&kv_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+    }
     for (int i = 0; i < C::kQStages; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
@@ -409,7 +433,6 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
     mbar_init(kv_done, 1);
-    mbar_init(kv_empty, 1);
     mbar_init(acc_empty, 128);
     mbar_init(mma_idle, 1);
     *abort_flag = 0;
@@ -423,16 +446,18 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+#ifdef FA_TRACE
   if (threadIdx.x == 0) {
     FA_TRACE_AT(6, 0, 0);
     uint32_t smid;
     asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
     int items = 0;
-    for (int u = 0; u < nunits; ++u) items += unit(u).total;
+    for (Job J = job0; J.gs < nslots; J = job_next(J)) items += unit(J).total;
     FA_TRACE_CTA(0, smid);
     FA_TRACE_CTA(1, items);
     FA_TRACE_CTA(2, globaltimer_ns());
   }
+#endif
 
   if (warp >= 12) {
     regs_dec<kBwdRegsOther>();
@@ -442,27 +467,32 @@ __global__ void __launch_bounds__(512, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       const bool stall = g_debug_stall != 0;  // test hook: the first K/V never arrive
-      int issued[C::kQStages];
+      int issued[C::kQStages], kv_issued[C::kKvBufs];
 #pragma unroll
       for (int i = 0; i < C::kQStages; ++i) issued[i] = 0;
-      int kv_loaded = 0, git = 0;
+#pragma unroll
+      for (int i = 0; i < C::kKvBufs; ++i) kv_issued[i] = 0;
+      int git = 0, u = 0;
       bool ok = true;
-      for (int u = 0; ok && u < nunits; ++u) {
-        const Unit U = unit(u);
-        // K and V of this unit replace the previous unit's once its products are done with them
-        if (u > 0 && !(ok = mbar_wait(kv_empty, (u - 1) & 1, abort_flag))) break;
+      for (Job J = job0; ok && J.gs < nslots; J = job_next(J), ++u) {
+        const Unit U = unit(J);
+        const int kb = u % C::kKvBufs;
+        // K and V of this job replace those of job u - kKvBufs once its products are done with them
+        if (u >= C::kKvBufs && !(ok = mbar_wait(&kv_empty[kb], (u / C::kKvBufs - 1) & 1, abort_flag))) break;
         if (!(stall && u == 0)) {
-          mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+          uint8_t* sK = sKV + kb * 2 * C::kTileBytes;
+          uint8_t* sV = sK + C::kTileBytes;
+          mbar_arrive_expect_tx(&kv_full[kb], 2 * C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided) {
-              tma_load_tile(&tmK, p.map4 & kBMapK, kv_full, sK + c * 16384, c * 64, U.k0, bkv, kh, b);
-              tma_load_tile(&tmV, p.map4 & kBMapV, kv_full, sV + c * 16384, c * 64, U.k0, bkv, kh, b);
+              tma_load_tile(&tmK, p.map4 & kBMapK, &kv_full[kb], sK + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
+              tma_load_tile(&tmV, p.map4 & kBMapV, &kv_full[kb], sV + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
             } else {
-              tma_load_3d(&tmK, kv_full, sK + c * 16384, c * 64, U.k0, bkv);
-              tma_load_3d(&tmV, kv_full, sV + c * 16384, c * 64, U.k0, bkv);
+              tma_load_3d(&tmK, &kv_full[kb], sK + c * 16384, c * 64, U.k0, U.bkv);
+              tma_load_3d(&tmV, &kv_full[kb], sV + c * 16384, c * 64, U.k0, U.bkv);
             }
           }
-          kv_loaded = u + 1;
+          ++kv_issued[kb];
         }
         QCursor cur = first(U);
         for (int it = 0; it < U.total; ++it, ++git, cur = advance(U, cur)) {
@@ -470,12 +500,12 @@ __global__ void __launch_bounds__(512, 1)
           if (!(ok = mbar_wait(&q_empty[s], ((git / C::kQStages) & 1) ^ 1, abort_flag))) break;
           FA_TRACE_AT(5, git, 0);
           mbar_arrive_expect_tx(&q_full[s], C::kTileBytes + C::kVecBytes);
-          const int row0 = cur.i * 128, bh = bh0 + cur.hq;
+          const int row0 = cur.i * 128, bh = U.bh0 + cur.hq;
           uint8_t* st = sQ + s * C::kTileBytes;
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided)
               tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, row0, bh,
-                            kh * p.g + cur.hq, b);
+                            U.kh * p.g + cur.hq, U.b);
             else
               tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
           }
@@ -486,7 +516,8 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
       // Never leave the CTA with copies still landing in shared memory.
-      if (kv_loaded > 0) mbar_wait_drain(kv_full, (kv_loaded - 1) & 1);
+      for (int kb = 0; kb < C::kKvBufs; ++kb)
+        if (kv_issued[kb] > 0) mbar_wait_drain(&kv_full[kb], (kv_issued[kb] - 1) & 1);
       for (int s = 0; s < C::kQStages; ++s)
         if (issued[s] > 0) mbar_wait_drain(&q_full[s], (issued[s] - 1) & 1);
     } else if (warp == 15 && lane == 0) {
@@ -497,20 +528,20 @@ __global__ void __launch_bounds__(512, 1)
       for (int i = 0; i < C::kDoStages; ++i) issued[i] = 0;
       int git = 0;
       bool ok = true;
-      for (int u = 0; ok && u < nunits; ++u) {
-        const Unit U = unit(u);
+      for (Job J = job0; ok && J.gs < nslots; J = job_next(J)) {
+        const Unit U = unit(J);
         QCursor cur = first(U);
         for (int it = 0; it < U.total; ++it, ++git, cur = advance(U, cur)) {
           const int s = git % C::kDoStages;
           if (!(ok = mbar_wait(&do_empty[s], ((git / C::kDoStages) & 1) ^ 1, abort_flag))) break;
           FA_TRACE_AT(5, git, 1);
           mbar_arrive_expect_tx(&do_full[s], C::kTileBytes);
-          const int row0 = cur.i * 128, bh = bh0 + cur.hq;
+          const int row0 = cur.i * 128, bh = U.bh0 + cur.hq;
           uint8_t* st = sDO + s * C::kTileBytes;
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided)
               tma_load_tile(&tmdO, p.map4 & kBMapDO, &do_full[s], st + c * 16384, c * 64, row0, bh,
-                            kh * p.g + cur.hq, b);
+                            U.kh * p.g + cur.hq, U.b);
             else
               tma_load_3d(&tmdO, &do_full[s], st + c * 16384, c * 64, row0, bh);
           }
@@ -527,8 +558,7 @@ __global__ void __launch_bounds__(512, 1)
       // dV and the next S^T then run while the compute warps form dS, and the
       // next dP^T is never queued behind them.  The chain runs on from one unit
       // into the next.
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), aDO = smem_u32(sDO),
-                     aDS = smem_u32(sDS);
+      const uint32_t aKV = smem_u32(sKV), aQ = smem_u32(sQ), aDO = smem_u32(sDO), aDS = smem_u32(sDS);
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdG = idesc_bf16_f32(128, D, false, true);     // dV, dK (A from TMEM)
       constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, true, true);      // dQ = dS K
@@ -550,10 +580,13 @@ __global__ void __launch_bounds__(512, 1)
                   sdesc_sw128(bb + k * 2048, 16384, 1024), kIdG, acc || k > 0);
       };
       bool ok = true;
-      int git = 0;  // work items of the CTA before the current one (barrier phases run on across units)
-      for (int u = 0; ok && u < nunits; ++u) {
-        const Unit U = unit(u);
-        if (!(ok = mbar_wait(kv_full, u & 1, abort_flag))) break;
+      int git = 0;  // work items of the CTA before the current one (barrier phases run on across jobs)
+      int u = 0;    // jobs of the CTA before the current one
+      for (Job J = job0; ok && J.gs < nslots; J = job_next(J), ++u) {
+        const Unit U = unit(J);
+        const int kb = u % C::kKvBufs;
+        const uint32_t aK = aKV + kb * 2 * C::kTileBytes, aV = aK + C::kTileBytes;
+        if (!(ok = mbar_wait(&kv_full[kb], (u / C::kKvBufs) & 1, abort_flag))) break;
         if (U.total > 0) {
           if (!(ok = mbar_wait(&q_full[git % C::kQStages], (git / C::kQStages) & 1, abort_flag))) break;
           tc_fence_after();
@@ -623,8 +656,8 @@ __global__ void __launch_bounds__(512, 1)
           if (!(ok = mbar_wait(acc_empty, (u - 1) & 1, abort_flag))) break;
         }
         git += U.total;
-        umma_commit(kv_empty);  // K and V may be replaced once these products complete
-        umma_commit(kv_done);   // dV and dK of the unit are complete
+        umma_commit(&kv_empty[kb]);  // K and V may be replaced once these products complete
+        umma_commit(kv_done);        // dV and dK of the job are complete
       }
       // Before the CTA frees TMEM: every product this thread issued has completed.
       umma_commit(mma_idle);
@@ -644,11 +677,11 @@ __global__ void __launch_bounds__(512, 1)
     const int ds_chunk = w;  // 64-column (128-byte) block of the dS tile
     bool ok = true;
     int git = 0;
-    for (int u = 0; ok && u < nunits; ++u) {
-      const Unit U = unit(u);
+    for (Job J = job0; ok && J.gs < nslots; J = job_next(J)) {
+      const Unit U = unit(J);
       const int key = U.k0 + r;
-      const bool tile_valid = U.k0 + 127 < Lb;  // no padded key in this key tile
-      const bool key_valid = key < Lb;
+      const bool tile_valid = U.k0 + 127 < U.Lb;  // no padded key in this key tile
+      const bool key_valid = key < U.Lb;
       QCursor cur = first(U);
       for (int it = 0; it < U.total; ++it, cur = advance(U, cur)) {
         const int g = git + it;
@@ -756,9 +789,9 @@ __global__ void __launch_bounds__(512, 1)
     constexpr int kBarDrain = 1, kBarDrainAnd = 2;  // named barriers of the 128 drain threads
     bool ok = true;
     int nchunk = 0;  // chunks handed to the TMA unit so far
-    int git = 0;
-    for (int u = 0; ok && u < nunits; ++u) {
-      const Unit U = unit(u);
+    int git = 0, u = 0;
+    for (Job J = job0; ok && J.gs < nslots; J = job_next(J), ++u) {
+      const Unit U = unit(J);
       QCursor cur = first(U);
       for (int it = 0; it < U.total; ++it, cur = advance(U, cur)) {
         const int g = git + it;
@@ -775,7 +808,7 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_before();
         mbar_arrive(dq_empty);  // TMEM tile free before the reductions are staged
         if (r == 0) FA_TRACE_AT(4, g, 1);
-        const size_t bh = static_cast<size_t>(bh0 + cur.hq);
+        const size_t bh = static_cast<size_t>(U.bh0 + cur.hq);
 #pragma unroll
         for (int c = 0; c < C::kDqChunks; ++c, ++nchunk) {
           uint8_t* buf = sDQ + (nchunk % C::kDqStages) * C::kDqChunkBytes;
@@ -836,9 +869,9 @@ __global__ void __launch_bounds__(512, 1)
       if (r == 0) {
         for (int c = 0; c < C::kChunks; ++c) {
           if constexpr (kStrided)
-            tma_store_tile(&tmdV, p.map4 & kBMapDV, sDV + c * 16384, c * 64, U.k0, bkv, kh, b);
+            tma_store_tile(&tmdV, p.map4 & kBMapDV, sDV + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
           else
-            tma_store_3d(&tmdV, sDV + c * 16384, c * 64, U.k0, bkv);
+            tma_store_3d(&tmdV, sDV + c * 16384, c * 64, U.k0, U.bkv);
         }
         bulk_commit();
         if (D == 128) bulk_wait_read0();  // dK reuses the buffers dV's store reads
@@ -852,9 +885,9 @@ __global__ void __launch_bounds__(512, 1)
       if (r == 0) {
         for (int c = 0; c < C::kChunks; ++c) {
           if constexpr (kStrided)
-            tma_store_tile(&tmdK, p.map4 & kBMapDK, sDK + c * 16384, c * 64, U.k0, bkv, kh, b);
+            tma_store_tile(&tmdK, p.map4 & kBMapDK, sDK + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
           else
-            tma_store_3d(&tmdK, sDK + c * 16384, c * 64, U.k0, bkv);
+            tma_store_3d(&tmdK, sDK + c * 16384, c * 64, U.k0, U.bkv);
         }
         bulk_commit();
         bulk_wait_read0();  // the next unit's dQ chunks reuse the staging buffers

@@ -187,6 +187,19 @@ fa_status check_strides(const fa::Strides& s, int B, int heads, int N, int d, in
   return FA_OK;
 }
 
+// Streaming multiprocessors of the current device (queried once per device);
+// 0 if the query fails.
+int sm_count() {
+  static std::mutex mu;
+  static int count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (count[dev] == 0 && cudaDeviceGetAttribute(&count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    count[dev] = 0;
+  return count[dev];
+}
+
 // Raises a kernel's dynamic shared-memory limit, once per (kernel, device):
 // the raised limits are remembered by kernel address and device.
 template <typename K>
@@ -487,7 +500,13 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
     return FA_ERR_CUDA;
   const size_t rows = static_cast<size_t>(B) * H * p.Np;
   const unsigned pre_grid = static_cast<unsigned>((rows + 8 * fa::kPreRowsPerWarp - 1) / (8 * fa::kPreRowsPerWarp));
-  const unsigned grid = static_cast<unsigned>(p.slots) * B * Hkv;
+  // Persistent: at most one CTA per SM, each running every gridDim-th slot.
+  // Block-sparse slots differ in work, so there every slot keeps its own CTA
+  // and the hardware balances them.
+  const unsigned nslots = static_cast<unsigned>(p.slots) * B * Hkv;
+  const int sms = sm_count();
+  if (sms <= 0) return FA_ERR_CUDA;
+  const unsigned grid = bmask ? nslots : std::min(nslots, static_cast<unsigned>(sms));
   const unsigned dq_grid = static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32));
   if (L) {
     if (bmask) return FA_ERR_UNSUPPORTED;
