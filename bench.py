@@ -18,6 +18,7 @@ on rank 0 only.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -536,6 +537,79 @@ def run_decode(args, rank, local):
     return 0
 
 
+PACKED_SHAPE = dict(H=16, Hkv=16, d=128, lo=64, hi=448)  # lengths uniform in [lo, hi], mean 256
+
+
+def packed_lengths(nseq: int, seed: int = 91):
+    """Seeded sequence lengths of the packed workload (uniform in [lo, hi])."""
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    return rng.integers(PACKED_SHAPE["lo"], PACKED_SHAPE["hi"] + 1, size=nseq).tolist()
+
+
+def run_packed(args, rank, local):
+    """Packed variable lengths (fa_fwd_packed / fa_bwd_packed): args.packed
+    short causal sequences concatenated along the token axis, forward +
+    backward per step, every sequence in one launch per kernel.  Flops are
+    counted per sequence as for the headline metric (4 L^2 d / 2 per head
+    forward, 2.5 times that backward)."""
+    import torch
+    import exact_io_aware_online_b200 as fa
+    from exact_io_aware_online_b200 import _build
+    if rank == 0:
+        _build.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    S = PACKED_SHAPE
+    H, Hkv, d = S["H"], S["Hkv"], S["d"]
+    lens = packed_lengths(args.packed)
+    cu = [0]
+    for L in lens:
+        cu.append(cu[-1] + L)
+    T = cu[-1]
+    g = torch.Generator("cpu").manual_seed(92 + rank)
+    q = torch.randn((T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    k = torch.randn((T, Hkv, d), generator=g).to(torch.bfloat16).to(dev)
+    v = torch.randn((T, Hkv, d), generator=g).to(torch.bfloat16).to(dev)
+    do = torch.randn((T, H, d), generator=g).to(torch.bfloat16).to(dev)
+    cu_dev = torch.tensor(cu, dtype=torch.int32, device=dev)
+    o, lse = torch.empty_like(q), torch.empty(T * H, dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    ws = torch.empty(int(fa.lib().fa_bwd_packed_workspace_size((ctypes.c_int * len(cu))(*cu), len(lens), H, d, 0)),
+                     dtype=torch.uint8, device=dev)
+    scale = 1.0 / d ** 0.5
+
+    def step():
+        fa.fwd_packed(q, k, v, cu_dev, scale, True, out=o, lse=lse)
+        fa.bwd_packed(q, k, v, o, lse, do, cu_dev, scale, True, workspace=ws, grads=grads)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    stream = torch.cuda.current_stream(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t0.record(stream)
+        for _ in range(K):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if fa.device_status() != 0:
+        raise RuntimeError("device-side timeout during the timed region")
+    ms = t0.elapsed_time(t1) / K
+    flops = sum(3.5 * 2.0 * L * L * d * H for L in lens)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "packed variable-length attention fwd+bwd TFLOP/s (bf16, causal, d=128)",
+            "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "n_gpus": 1, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"packed_{len(lens)}seq_len{S['lo']}to{S['hi']}_h{H}_d{d}_causal", "tokens": T,
+                       "l2": f"{4 * T * H * d * 2 / 2**20:.0f} MiB of Q, K, V, dO per step (no flush)"},
+            "clocks": clk.summary(), "gpu_launches": 4 * K}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -554,6 +628,9 @@ def main():
     ap.add_argument("--decode", type=int, default=0,
                     help="time the decode forward instead: this many new queries per sequence against a "
                          "32768-token cache (B=8, 32 query heads on 8 kv heads, d=128, causal)")
+    ap.add_argument("--packed", type=int, default=0,
+                    help="time packed variable lengths instead: this many causal sequences of 64..448 tokens "
+                         "(16 heads, d=128), forward + backward, one launch per kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -570,6 +647,10 @@ def main():
             if world > 1 or args.impl != "ours":
                 raise SystemExit("--decode: one GPU, --impl ours only")
             return run_decode(args, rank, local)
+        if args.packed:
+            if world > 1 or args.impl != "ours":
+                raise SystemExit("--packed: one GPU, --impl ours only")
+            return run_packed(args, rank, local)
         if args.impl == "reference":
             return run_reference(args, w, world, rank)
         return run_ours(args, w, world, rank, local)

@@ -92,7 +92,43 @@ struct BwdParams {
 struct BwdStridedParams : BwdParams {
   Strides so, sdo, sdq;
   unsigned map4;
+  // Packed variable lengths (non-null rowoff, device memory): batch entry b is
+  // sequence b, rows rowoff[b] .. rowoff[b+1] - 1 of tensors that hold all T
+  // rows back to back (one batch entry in the tensor maps and strides); N is
+  // the longest length.  The workspace rows of sequence b start at
+  // packed_ws_row(b) inside each head's tp rows; the logsumexp of sequence b is
+  // [H, len_b] at lse + rowoff[b] * H; dK and dV rows are stored only up to the
+  // sequence end (plain stores for a key tile the end falls inside).
+  const int* rowoff;
+  int T;
+  int tp;  // workspace rows per head: 128 * (ceil(T / 128) + B)
+  void* dk;
+  void* dv;
+  long long kv_rs, kv_hs;  // element strides of dK / dV rows and heads
 };
+// First workspace row of packed sequence b (a multiple of 128): consecutive
+// sequences' padded row ranges [start, start + 128 * ceil(len / 128)) never
+// overlap, since floor(rowoff[b + 1] / 128) >= floor(rowoff[b] / 128) +
+// floor(len_b / 128).
+__device__ __forceinline__ int packed_ws_row(int rowoff_b, int b) { return 128 * (rowoff_b / 128 + b); }
+// Sequence b's first row and length, clamped to the tensors' T rows.
+__device__ __forceinline__ void packed_range(const BwdStridedParams& p, int b, int& rb, int& len) {
+  rb = min(max(p.rowoff[b], 0), p.T);
+  len = min(min(max(p.rowoff[b + 1], rb), p.T) - rb, p.N);
+}
+// The packed sequence whose workspace rows hold row R (0 <= R < tp): the last b
+// with packed_ws_row(b) <= R (binary search; starts increase with b).
+__device__ __forceinline__ int packed_seq_of_ws_row(const BwdStridedParams& p, int R) {
+  int lo = 0, hi = p.B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (packed_ws_row(min(max(p.rowoff[mid], 0), p.T), mid) <= R)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
 constexpr unsigned kBMapQ = 1, kBMapK = 2, kBMapV = 4, kBMapDO = 8, kBMapDK = 16, kBMapDV = 32;
 template <bool kStrided>
 using BwdArgs = std::conditional_t<kStrided, BwdStridedParams, BwdParams>;
@@ -149,28 +185,44 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p)
   constexpr int kRowsPerPass = 32 / kLanesPerRow;  // 2 (D = 128) or 4 (D = 64)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / kLanesPerRow, part = lane % kLanesPerRow;
-  const size_t rows = static_cast<size_t>(p.B) * p.H * p.Np;
+  bool packed = false;
+  if constexpr (kStrided) packed = p.rowoff != nullptr;
+  // workspace rows: B*H*Np, or (packed) H*tp
+  size_t rows = static_cast<size_t>(p.B) * p.H * p.Np;
+  if constexpr (kStrided)
+    if (packed) rows = static_cast<size_t>(p.H) * p.tp;
   const size_t row0 = (static_cast<size_t>(blockIdx.x) * 8 + warp) * kPreRowsPerWarp;
 #pragma unroll
   for (int pass = 0; pass < kPreRowsPerWarp / kRowsPerPass; ++pass) {
-    const size_t row = row0 + pass * kRowsPerPass + sub;  // over B*H*Np
+    const size_t row = row0 + pass * kRowsPerPass + sub;  // over the workspace rows
     const bool in = row < rows;
-    const size_t bh = in ? row / p.Np : 0;
-    const int n = in ? static_cast<int>(row % p.Np) : 0;
+    size_t bh = in ? row / p.Np : 0;
+    int n = in ? static_cast<int>(row % p.Np) : 0;
+    int len = 0, rb = 0;  // packed: the sequence's length and first row
+    if constexpr (kStrided) {
+      if (packed && in) {
+        const int h = static_cast<int>(row / p.tp), R = static_cast<int>(row % p.tp);
+        const int b = packed_seq_of_ws_row(p, R);
+        packed_range(p, b, rb, len);
+        n = R - packed_ws_row(rb, b);
+        bh = static_cast<size_t>(b) * p.H + h;
+      }
+    }
     if (in) {  // zero D floats of the dQ accumulator (every float is zeroed once, whatever the layout)
       float4* acc = reinterpret_cast<float4*>(p.dqacc + row * D);
       acc[2 * part] = make_float4(0.f, 0.f, 0.f, 0.f);
       acc[2 * part + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    const bool valid = in && n < valid_rows(p, static_cast<int>(bh / p.H));
+    const bool valid = in && n >= 0 && n < (packed ? len : valid_rows(p, static_cast<int>(bh / p.H)));
     float s = 0.f;
     if (valid) {
       const __nv_bfloat16* orow;
       const __nv_bfloat16* drow;
       if constexpr (kStrided) {
         const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
-        orow = static_cast<const __nv_bfloat16*>(p.o) + p.so.row(b, h, n);
-        drow = static_cast<const __nv_bfloat16*>(p.dout) + p.sdo.row(b, h, n);
+        const int bi = packed ? 0 : b, ni = packed ? rb + n : n;  // packed: one batch entry of T rows
+        orow = static_cast<const __nv_bfloat16*>(p.o) + p.so.row(bi, h, ni);
+        drow = static_cast<const __nv_bfloat16*>(p.dout) + p.sdo.row(bi, h, ni);
       } else {
         orow = static_cast<const __nv_bfloat16*>(p.o) + (bh * p.N + n) * D;
         drow = static_cast<const __nv_bfloat16*>(p.dout) + (bh * p.N + n) * D;
@@ -188,8 +240,13 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p)
     for (int off = kLanesPerRow / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (in && part == 0) {
       // tile padding or a padded token: D = 0 and LSE = +inf, so its P is exactly 0
+      float lse = 0.f;
+      if (valid) {
+        const size_t h = bh % p.H;
+        lse = packed ? p.lse[static_cast<size_t>(rb) * p.H + h * len + n] : p.lse[bh * p.N + n];
+      }
       p.nD[row] = valid ? -s : 0.f;
-      p.nlse2[row] = valid ? -p.lse[bh * p.N + n] * 1.4426950408889634f : -INFINITY;
+      p.nlse2[row] = valid ? -lse * 1.4426950408889634f : -INFINITY;
     }
   }
 }
@@ -214,15 +271,35 @@ __device__ __forceinline__ size_t dqacc_chunk(size_t bh, int ntiles, int tile, i
 template <int D, bool kStrided = false>
 __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs<kStrided> p) {
   __shared__ float tile[32][D + 4];
-  const int groups = p.Np / 32;
-  const size_t bh = blockIdx.x / groups;
+  // One block per 32 workspace rows: of head bh's Np rows, or (packed) of head
+  // h's tp rows, where they belong to sequence b (rows past its end are skipped).
+  int groups = p.Np / 32;
+  bool packed = false;
+  if constexpr (kStrided) {
+    packed = p.rowoff != nullptr;
+    if (packed) groups = p.tp / 32;
+  }
+  size_t bh = blockIdx.x / groups;
   const int g = static_cast<int>(blockIdx.x % groups);
+  size_t tile0 = bh * p.ntiles;  // the accumulator's first 128-row tile of this head
+  int nbase = 32 * g, nend = p.N, nvalid = 0, rb = 0;  // first row of the group, row limit, valid rows
+  if constexpr (kStrided) {
+    if (packed) {
+      const int h = static_cast<int>(bh), b = packed_seq_of_ws_row(p, 32 * g);
+      packed_range(p, b, rb, nvalid);
+      nbase = 32 * g - packed_ws_row(rb, b);
+      nend = nvalid;
+      tile0 = static_cast<size_t>(h) * (p.tp / 128);
+      bh = static_cast<size_t>(b) * p.H + h;
+    }
+  }
+  if (!packed) nvalid = valid_rows(p, static_cast<int>(bh / p.H));
   const int t128 = g >> 2, r0 = (g & 3) * 32;  // 128-row tile and first row inside it
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {  // 32 rows x 8 units of one chunk: 256 float4, one per thread
     const int rr = threadIdx.x >> 3, up = threadIdx.x & 7;
     const int u = up ^ (rr & 7);  // r0 is a multiple of 8, so (r0 + rr) % 8 = rr % 8
-    const float4 a = reinterpret_cast<const float4*>(p.dqacc + dqacc_chunk<D>(bh, p.ntiles, t128, c) +
+    const float4 a = reinterpret_cast<const float4*>(p.dqacc + ((tile0 + t128) * (D / 32) + c) * 4096 +
                                                      static_cast<size_t>(r0) * 32)[threadIdx.x];
     *reinterpret_cast<float4*>(&tile[rr][c * 32 + 4 * u]) = a;
   }
@@ -231,15 +308,16 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs<kStrided> p) 
   for (int k = 0; k < D / 32; ++k) {
     const int f = threadIdx.x + 256 * k;
     const int rr = f / (D / 4), u = f % (D / 4);
-    const int n = 32 * g + rr;
-    if (n >= p.N) continue;
-    const float sc = n < valid_rows(p, static_cast<int>(bh / p.H)) ? p.scale : 0.f;
+    const int n = nbase + rr;
+    if (n < 0 || n >= nend) continue;
+    const float sc = n < nvalid ? p.scale : 0.f;
     uint2 out;
     out.x = pack_bf16x2(tile[rr][4 * u + 0] * sc, tile[rr][4 * u + 1] * sc);
     out.y = pack_bf16x2(tile[rr][4 * u + 2] * sc, tile[rr][4 * u + 3] * sc);
     long long at;
     if constexpr (kStrided)
-      at = p.sdq.row(static_cast<int>(bh / p.H), static_cast<int>(bh % p.H), n) + 4 * u;
+      at = packed ? p.sdq.row(0, static_cast<int>(bh % p.H), rb + n) + 4 * u
+                  : p.sdq.row(static_cast<int>(bh / p.H), static_cast<int>(bh % p.H), n) + 4 * u;
     else
       at = static_cast<long long>((bh * p.N + n) * D + 4 * u);
     *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + at) = out;
@@ -366,7 +444,14 @@ __global__ void __launch_bounds__(512, 1)
   struct Unit {
     int j, k0, ilo, ihi, total;
     int bkv, b, kh, bh0, Lb;  // kv head, batch entry, kv head in it, first query head, valid rows
+    int rb, cb, ckv, cq0;     // tensor-map coordinates: first row, batch entry, kv head, first query head
+    size_t w0;                // workspace row of (first query head, row 0); query head hq adds hq * wstride
   };
+  bool packed = false;
+  if constexpr (kStrided) packed = p.rowoff != nullptr;
+  size_t wstride = p.Np;  // workspace rows per query head
+  if constexpr (kStrided)
+    if (packed) wstride = p.tp;
   struct QCursor {
     int hq, i;
   };
@@ -395,6 +480,20 @@ __global__ void __launch_bounds__(512, 1)
     U.kh = U.bkv % p.Hkv;
     U.Lb = valid_rows(p, U.b);
     U.bh0 = U.b * p.H + U.kh * p.g;
+    U.rb = 0;
+    U.cb = U.b;
+    U.ckv = U.bkv;
+    U.cq0 = U.bh0;
+    U.w0 = static_cast<size_t>(U.bh0) * p.Np;
+    if constexpr (kStrided) {
+      if (packed) {  // one batch entry of T rows in the maps; the sequence starts at row rb
+        packed_range(p, U.b, U.rb, U.Lb);
+        U.cb = 0;
+        U.ckv = U.kh;
+        U.cq0 = U.kh * p.g;
+        U.w0 = static_cast<size_t>(U.kh * p.g) * p.tp + packed_ws_row(U.rb, U.b);
+      }
+    }
     U.j = p.pairs ? (J.sub == 0 ? slot : p.ntiles - 1 - slot) : slot;
     U.k0 = U.j * 128;
     U.ilo = 0;
@@ -485,8 +584,10 @@ __global__ void __launch_bounds__(512, 1)
           mbar_arrive_expect_tx(&kv_full[kb], 2 * C::kTileBytes);
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided) {
-              tma_load_tile(&tmK, p.map4 & kBMapK, &kv_full[kb], sK + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
-              tma_load_tile(&tmV, p.map4 & kBMapV, &kv_full[kb], sV + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
+              tma_load_tile(&tmK, p.map4 & kBMapK, &kv_full[kb], sK + c * 16384, c * 64, U.rb + U.k0, U.ckv, U.kh,
+                            U.cb);
+              tma_load_tile(&tmV, p.map4 & kBMapV, &kv_full[kb], sV + c * 16384, c * 64, U.rb + U.k0, U.ckv, U.kh,
+                            U.cb);
             } else {
               tma_load_3d(&tmK, &kv_full[kb], sK + c * 16384, c * 64, U.k0, U.bkv);
               tma_load_3d(&tmV, &kv_full[kb], sV + c * 16384, c * 64, U.k0, U.bkv);
@@ -504,12 +605,12 @@ __global__ void __launch_bounds__(512, 1)
           uint8_t* st = sQ + s * C::kTileBytes;
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided)
-              tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, row0, bh,
-                            U.kh * p.g + cur.hq, U.b);
+              tma_load_tile(&tmQ, p.map4 & kBMapQ, &q_full[s], st + c * 16384, c * 64, U.rb + row0, U.cq0 + cur.hq,
+                            U.kh * p.g + cur.hq, U.cb);
             else
               tma_load_3d(&tmQ, &q_full[s], st + c * 16384, c * 64, row0, bh);
           }
-          const size_t vrow = static_cast<size_t>(bh) * p.Np + row0;
+          const size_t vrow = U.w0 + cur.hq * wstride + row0;
           bulk_load(sVec + s * C::kVecBytes, p.nlse2 + vrow, 512, &q_full[s]);
           bulk_load(sVec + s * C::kVecBytes + 512, p.nD + vrow, 512, &q_full[s]);
           ++issued[s];
@@ -540,8 +641,8 @@ __global__ void __launch_bounds__(512, 1)
           uint8_t* st = sDO + s * C::kTileBytes;
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided)
-              tma_load_tile(&tmdO, p.map4 & kBMapDO, &do_full[s], st + c * 16384, c * 64, row0, bh,
-                            U.kh * p.g + cur.hq, U.b);
+              tma_load_tile(&tmdO, p.map4 & kBMapDO, &do_full[s], st + c * 16384, c * 64, U.rb + row0,
+                            U.cq0 + cur.hq, U.kh * p.g + cur.hq, U.cb);
             else
               tma_load_3d(&tmdO, &do_full[s], st + c * 16384, c * 64, row0, bh);
           }
@@ -808,7 +909,8 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_before();
         mbar_arrive(dq_empty);  // TMEM tile free before the reductions are staged
         if (r == 0) FA_TRACE_AT(4, g, 1);
-        const size_t bh = static_cast<size_t>(U.bh0 + cur.hq);
+        // the accumulator's 128-row tiles of this query head (dqacc_chunk's order)
+        const size_t tile0 = (U.w0 + cur.hq * wstride) / 128;
 #pragma unroll
         for (int c = 0; c < C::kDqChunks; ++c, ++nchunk) {
           uint8_t* buf = sDQ + (nchunk % C::kDqStages) * C::kDqChunkBytes;
@@ -823,7 +925,7 @@ __global__ void __launch_bounds__(512, 1)
           fence_proxy_async_smem();
           named_bar_sync(kBarDrain, 128);
           if (r == 0) {
-            bulk_reduce_add_f32(p.dqacc + dqacc_chunk<D>(bh, p.ntiles, cur.i, c), buf, C::kDqChunkBytes);
+            bulk_reduce_add_f32(p.dqacc + ((tile0 + cur.i) * (D / 32) + c) * 4096, buf, C::kDqChunkBytes);
             bulk_commit();
           }
         }
@@ -839,6 +941,25 @@ __global__ void __launch_bounds__(512, 1)
       named_bar_sync(kBarDrain, 128);
       uint8_t* sDV = sDQ;                                  // bf16 128 x D tile in the TMA layout
       uint8_t* sDK = sDQ + (D == 128 ? 0 : C::kTileBytes);  // after dV's store has read it (D = 128)
+      // Stores: the whole tile by the TMA unit, or (packed, the sequence ends
+      // inside the key tile) each valid row by its own thread, or (packed, the
+      // tile lies past the sequence end) nothing.
+      const bool tma_out = !packed || U.k0 + 128 <= U.Lb;
+      auto store_rows = [&](const uint8_t* sT, bool is_dk) {  // my row of a staged tile, if valid
+        if constexpr (kStrided) {
+          if (U.k0 + r < U.Lb) {
+            __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(is_dk ? p.dk : p.dv) +
+                                 static_cast<long long>(U.rb + U.k0 + r) * p.kv_rs +
+                                 static_cast<long long>(U.kh) * p.kv_hs;
+#pragma unroll
+            for (int cc = 0; cc < D / 64; ++cc)
+#pragma unroll
+              for (int u8 = 0; u8 < 8; ++u8)
+                *reinterpret_cast<uint4*>(dst + cc * 64 + u8 * 8) =
+                    *reinterpret_cast<const uint4*>(sT + cc * 16384 + r * 128 + ((u8 ^ (r & 7)) << 4));
+          }
+        }
+      };
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t t[32];
@@ -866,32 +987,34 @@ __global__ void __launch_bounds__(512, 1)
       mbar_arrive(acc_empty);  // the next unit's products may overwrite dV and dK
       fence_proxy_async_smem();
       named_bar_sync(kBarDrain, 128);
-      if (r == 0) {
+      if (r == 0 && tma_out) {
         for (int c = 0; c < C::kChunks; ++c) {
           if constexpr (kStrided)
-            tma_store_tile(&tmdV, p.map4 & kBMapDV, sDV + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
+            tma_store_tile(&tmdV, p.map4 & kBMapDV, sDV + c * 16384, c * 64, U.rb + U.k0, U.ckv, U.kh, U.cb);
           else
             tma_store_3d(&tmdV, sDV + c * 16384, c * 64, U.k0, U.bkv);
         }
         bulk_commit();
         if (D == 128) bulk_wait_read0();  // dK reuses the buffers dV's store reads
       }
+      if (!tma_out) store_rows(sDV, false);
       named_bar_sync(kBarDrain, 128);
 #pragma unroll
       for (int c = 0; c < D; c += 32)
         stage_row32_bf16(sDK, r, c, *reinterpret_cast<const uint32_t(*)[32]>(&v[c]), p.scale);
       fence_proxy_async_smem();
       named_bar_sync(kBarDrain, 128);
-      if (r == 0) {
+      if (r == 0 && tma_out) {
         for (int c = 0; c < C::kChunks; ++c) {
           if constexpr (kStrided)
-            tma_store_tile(&tmdK, p.map4 & kBMapDK, sDK + c * 16384, c * 64, U.k0, U.bkv, U.kh, U.b);
+            tma_store_tile(&tmdK, p.map4 & kBMapDK, sDK + c * 16384, c * 64, U.rb + U.k0, U.ckv, U.kh, U.cb);
           else
             tma_store_3d(&tmdK, sDK + c * 16384, c * 64, U.k0, U.bkv);
         }
         bulk_commit();
         bulk_wait_read0();  // the next unit's dQ chunks reuse the staging buffers
       }
+      if (!tma_out) store_rows(sDK, true);
       named_bar_sync(kBarDrain, 128);
     }
     // Shared memory must outlive the copies that read it; the global side of the

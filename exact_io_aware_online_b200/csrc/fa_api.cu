@@ -16,7 +16,7 @@
 
 namespace {
 
-constexpr int kAbiVersion = 100;
+constexpr int kAbiVersion = 101;
 
 cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;  // fa_set_timing_events
 inline void mark_start(cudaStream_t st) {
@@ -137,6 +137,13 @@ bool make_tile_map(CUtensorMap* m, const void* ptr, int B, int heads, int N, int
 // Element strides of every tensor argument of one call.
 struct Layouts {
   fa::Strides q, k, v, o, dout, dq, dk, dv;
+};
+
+// Packed variable lengths in one launch: the B sequences' offsets (device
+// copy, read by the kernels) and the total row count T of the packed tensors.
+struct Packed {
+  const int* rowoff;
+  int T;
 };
 
 Layouts contiguous_layouts(int B, int H, int Hkv, int N, int d) {
@@ -267,14 +274,16 @@ template <int D>
 fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv, int N,
                    float scale, int causal, int window, cudaStream_t st, const Layouts* L = nullptr, int splits = 0,
                    void* ws = nullptr, const uint8_t* bmask = nullptr, long long bmask_hs = 0,
-                   const int* seqlens = nullptr) {
+                   const int* seqlens = nullptr, const Packed* pk = nullptr) {
   fa_status ls = FA_OK;
   using C = fa::FwdCfg<D>;
   const Layouts lay = L ? *L : contiguous_layouts(B, H, Hkv, N, D);
   CUtensorMap tq, tk, tv, to;
   bool f4[4];
-  if (!make_tile_map(&tq, q, B, H, N, D, lay.q, &f4[0]) || !make_tile_map(&tk, k, B, Hkv, N, D, lay.k, &f4[1]) ||
-      !make_tile_map(&tv, v, B, Hkv, N, D, lay.v, &f4[2]) || !make_tile_map(&to, o, B, H, N, D, lay.o, &f4[3]))
+  // packed: the maps cover all T rows as one batch entry; N is the longest sequence
+  const int mB = pk ? 1 : B, mN = pk ? pk->T : N;
+  if (!make_tile_map(&tq, q, mB, H, mN, D, lay.q, &f4[0]) || !make_tile_map(&tk, k, mB, Hkv, mN, D, lay.k, &f4[1]) ||
+      !make_tile_map(&tv, v, mB, Hkv, mN, D, lay.v, &f4[2]) || !make_tile_map(&to, o, mB, H, mN, D, lay.o, &f4[3]))
     return FA_ERR_CUDA;
   if (!set_smem(fa::fwd_sm100_kernel<D, false, false>, C::kSmemBytes) ||
       !set_smem(fa::fwd_sm100_kernel<D, true, false>, C::kSmemBytes) ||
@@ -310,6 +319,13 @@ fa_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* 
     static_cast<fa::FwdParams&>(ps) = p;
     ps.map4 = (f4[0] ? fa::kMapQ : 0u) | (f4[1] ? fa::kMapK : 0u) | (f4[2] ? fa::kMapV : 0u) |
               (f4[3] ? fa::kMapO : 0u);
+    if (pk) {
+      ps.rowoff = pk->rowoff;
+      ps.T = pk->T;
+      ps.o = o;
+      ps.o_rs = lay.o.n;
+      ps.o_hs = lay.o.h;
+    }
     mark_start(st);
     ls = launch(fa::fwd_sm100_kernel<D, false, false, true>, grid, C::kThreads, C::kSmemBytes, st, tq, tk, tv, to, ps);
     mark_stop(st);
@@ -431,6 +447,9 @@ fa_status fwd_f32(const void* q, const void* k, const void* v, void* o, float* l
 struct WsLayout {
   size_t nlse2, nd, dqacc, total;
 };
+// Workspace rows per head of a packed backward: every sequence's rows padded to
+// whole 128-row tiles, at 128-aligned starts (packed_ws_row in the kernels).
+int packed_ws_rows(int T, int B) { return 128 * ((T + 127) / 128 + B); }
 WsLayout ws_layout(int B, int H, int N, int d, fa_dtype dtype) {
   WsLayout w{};
   if (dtype == FA_FP32) {
@@ -450,10 +469,12 @@ template <int D>
 fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                    void* dq, void* dk, void* dv, void* ws, int B, int H, int Hkv, int N, float scale, int causal,
                    int window, cudaStream_t st, const Layouts* L = nullptr, const uint8_t* bmask = nullptr,
-                   long long bmask_hs = 0, const int* seqlens = nullptr) {
+                   long long bmask_hs = 0, const int* seqlens = nullptr, const Packed* pk = nullptr) {
   fa_status ls = FA_OK;
   using C = fa::BwdCfg<D>;
-  const WsLayout w = ws_layout(B, H, N, D, FA_BF16);
+  // packed: each head's workspace rows hold every sequence's padded rows (tp of them)
+  const int tp = pk ? packed_ws_rows(pk->T, B) : 0;
+  const WsLayout w = pk ? ws_layout(1, H, tp, D, FA_BF16) : ws_layout(B, H, N, D, FA_BF16);
   const Layouts lay = L ? *L : contiguous_layouts(B, H, Hkv, N, D);
   uint8_t* wb = static_cast<uint8_t*>(ws);
   fa::BwdParams p{};
@@ -489,16 +510,18 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   }
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   bool f4[6];
-  if (!make_tile_map(&tq, q, B, H, N, D, lay.q, &f4[0]) || !make_tile_map(&tk, k, B, Hkv, N, D, lay.k, &f4[1]) ||
-      !make_tile_map(&tv, v, B, Hkv, N, D, lay.v, &f4[2]) ||
-      !make_tile_map(&tdo, dout, B, H, N, D, lay.dout, &f4[3]) ||
-      !make_tile_map(&tdk, dk, B, Hkv, N, D, lay.dk, &f4[4]) || !make_tile_map(&tdv, dv, B, Hkv, N, D, lay.dv, &f4[5]))
+  const int mB = pk ? 1 : B, mN = pk ? pk->T : N;  // packed: one batch entry of T rows
+  if (!make_tile_map(&tq, q, mB, H, mN, D, lay.q, &f4[0]) || !make_tile_map(&tk, k, mB, Hkv, mN, D, lay.k, &f4[1]) ||
+      !make_tile_map(&tv, v, mB, Hkv, mN, D, lay.v, &f4[2]) ||
+      !make_tile_map(&tdo, dout, mB, H, mN, D, lay.dout, &f4[3]) ||
+      !make_tile_map(&tdk, dk, mB, Hkv, mN, D, lay.dk, &f4[4]) ||
+      !make_tile_map(&tdv, dv, mB, Hkv, mN, D, lay.dv, &f4[5]))
     return FA_ERR_CUDA;
   if (!set_smem(fa::bwd_sm100_kernel<D, false>, C::kSmemBytes) ||
       !set_smem(fa::bwd_sm100_kernel<D, true>, C::kSmemBytes) ||
       !set_smem(fa::bwd_sm100_kernel<D, false, true>, C::kSmemBytes))
     return FA_ERR_CUDA;
-  const size_t rows = static_cast<size_t>(B) * H * p.Np;
+  const size_t rows = pk ? static_cast<size_t>(H) * tp : static_cast<size_t>(B) * H * p.Np;  // workspace rows
   const unsigned pre_grid = static_cast<unsigned>((rows + 8 * fa::kPreRowsPerWarp - 1) / (8 * fa::kPreRowsPerWarp));
   // Persistent: at most one CTA per SM, each running every gridDim-th slot.
   // Block-sparse slots differ in work, so there every slot keeps its own CTA
@@ -507,7 +530,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   const int sms = sm_count();
   if (sms <= 0) return FA_ERR_CUDA;
   const unsigned grid = bmask ? nslots : std::min(nslots, static_cast<unsigned>(sms));
-  const unsigned dq_grid = static_cast<unsigned>(static_cast<size_t>(B) * H * (p.Np / 32));
+  const unsigned dq_grid = static_cast<unsigned>(rows / 32);
   if (L) {
     if (bmask) return FA_ERR_UNSUPPORTED;
     fa::BwdStridedParams ps{};
@@ -517,6 +540,15 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
     ps.sdq = lay.dq;
     ps.map4 = (f4[0] ? fa::kBMapQ : 0u) | (f4[1] ? fa::kBMapK : 0u) | (f4[2] ? fa::kBMapV : 0u) |
               (f4[3] ? fa::kBMapDO : 0u) | (f4[4] ? fa::kBMapDK : 0u) | (f4[5] ? fa::kBMapDV : 0u);
+    if (pk) {
+      ps.rowoff = pk->rowoff;
+      ps.T = pk->T;
+      ps.tp = tp;
+      ps.dk = dk;
+      ps.dv = dv;
+      ps.kv_rs = lay.dk.n;
+      ps.kv_hs = lay.dk.h;
+    }
     ls = launch(fa::bwd_pre_kernel<D, true>, pre_grid, 256, 0, st, ps);
     if (ls != FA_OK) return ls;
     mark_start(st);
@@ -589,6 +621,13 @@ fa_status packed_lengths(const int* cu, int B, int* max_len) {
     m = std::max(m, cu[b + 1] - cu[b]);
   }
   *max_len = m;
+  return FA_OK;
+}
+
+// Packed tensors of T rows in one launch: the row count and the workspace rows
+// must stay within int range (tensor-map coordinates and kernel indices).
+fa_status check_packed_rows(int T, int B) {
+  if (T < 0 || static_cast<long long>(T) + 128LL * (B + 1) > (1LL << 30)) return FA_ERR_INVALID_ARG;
   return FA_OK;
 }
 
@@ -846,8 +885,8 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
 }
 
 fa_status fa_fwd_packed(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
-                        int B, int H, int Hkv, int d, float scale, int causal, int window, fa_dtype dtype,
-                        void* stream) {
+                        const int* cu_seqlens_dev, int B, int H, int Hkv, int d, float scale, int causal, int window,
+                        fa_dtype dtype, void* stream) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   int max_len = 0;
   fa_status s = packed_lengths(cu_seqlens, B, &max_len);
@@ -856,7 +895,22 @@ fa_status fa_fwd_packed(const void* q, const void* k, const void* v, void* o, fl
   if (s != FA_OK) return s;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_MISALIGNED;
   const size_t es = dtype == FA_BF16 ? 2 : 4;
-  for (int b = 0; b < B; ++b) {
+  const int T = cu_seqlens[B];
+  if (T == 0) return FA_OK;
+  if (dtype == FA_BF16) {  // one launch over every sequence
+    if (!cu_seqlens_dev || !aligned16(cu_seqlens_dev)) return FA_ERR_INVALID_ARG;
+    if ((s = check_packed_rows(T, B)) != FA_OK) return s;
+    Layouts L{};
+    if ((s = packed_layouts(H, Hkv, T, d, static_cast<int>(es), &L)) != FA_OK) return s;
+    if ((s = check_stream(stream)) != FA_OK) return s;
+    const Packed pk{cu_seqlens_dev, T};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return d == 64 ? fwd_bf16<64>(q, k, v, o, lse, B, H, Hkv, max_len, scale, causal, window, st, &L, 0, nullptr,
+                                  nullptr, 0, nullptr, &pk)
+                   : fwd_bf16<128>(q, k, v, o, lse, B, H, Hkv, max_len, scale, causal, window, st, &L, 0, nullptr,
+                                   nullptr, 0, nullptr, &pk);
+  }
+  for (int b = 0; b < B; ++b) {  // fp32: one launch per sequence
     const int len = cu_seqlens[b + 1] - cu_seqlens[b];
     if (len == 0) continue;
     Layouts L{};
@@ -875,24 +929,45 @@ size_t fa_bwd_packed_workspace_size(const int* cu_seqlens, int B, int H, int d, 
   int max_len = 0;
   if (packed_lengths(cu_seqlens, B, &max_len) != FA_OK) return 0;
   if (check_common(1, H, 1, std::max(max_len, 1), d, 1.0f, -1, dtype) != FA_OK) return 0;
+  if (dtype == FA_BF16) {
+    if (check_packed_rows(cu_seqlens[B], B) != FA_OK) return 0;
+    return ws_layout(1, H, packed_ws_rows(cu_seqlens[B], B), d, dtype).total;
+  }
   return ws_layout(1, H, std::max(max_len, 1), d, dtype).total;
 }
 
 fa_status fa_bwd_packed(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                        const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens, void* workspace,
-                        size_t ws_bytes, int B, int H, int Hkv, int d, float scale, int causal, int window,
-                        fa_dtype dtype, void* stream) {
+                        const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens,
+                        const int* cu_seqlens_dev, void* workspace, size_t ws_bytes, int B, int H, int Hkv, int d,
+                        float scale, int causal, int window, fa_dtype dtype, void* stream) {
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   int max_len = 0;
   fa_status s = packed_lengths(cu_seqlens, B, &max_len);
   if (s != FA_OK) return s;
   s = check_common(1, H, Hkv, std::max(max_len, 1), d, scale, window, dtype);
   if (s != FA_OK) return s;
+  const size_t need = fa_bwd_packed_workspace_size(cu_seqlens, B, H, d, dtype);
+  if (need == 0) return FA_ERR_INVALID_ARG;
   s = check_bwd_buffers(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, 1, H, std::max(max_len, 1), d,
                         dtype);
   if (s != FA_OK) return s;
+  if (ws_bytes < need) return FA_ERR_WORKSPACE;
   const size_t es = dtype == FA_BF16 ? 2 : 4;
-  for (int b = 0; b < B; ++b) {  // in stream order: each sequence reuses the workspace after the previous one
+  const int T = cu_seqlens[B];
+  if (T == 0) return FA_OK;
+  if (dtype == FA_BF16) {  // one launch of each backward kernel over every sequence
+    if (!cu_seqlens_dev || !aligned16(cu_seqlens_dev)) return FA_ERR_INVALID_ARG;
+    Layouts L{};
+    if ((s = packed_layouts(H, Hkv, T, d, static_cast<int>(es), &L)) != FA_OK) return s;
+    if ((s = check_stream(stream)) != FA_OK) return s;
+    const Packed pk{cu_seqlens_dev, T};
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return d == 64 ? bwd_bf16<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, max_len, scale, causal,
+                                  window, st, &L, nullptr, 0, nullptr, &pk)
+                   : bwd_bf16<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, max_len, scale, causal,
+                                   window, st, &L, nullptr, 0, nullptr, &pk);
+  }
+  for (int b = 0; b < B; ++b) {  // fp32: in stream order, each sequence reuses the workspace after the previous one
     const int len = cu_seqlens[b + 1] - cu_seqlens[b];
     if (len == 0) continue;
     Layouts L{};

@@ -66,6 +66,16 @@ struct FwdParams {
 // instantiations keep the plain FwdParams.
 struct FwdStridedParams : FwdParams {
   unsigned map4;
+  // Packed variable lengths (non-null rowoff, device memory): batch entry b is
+  // sequence b, rows rowoff[b] .. rowoff[b+1] - 1 of tensors that hold all T
+  // rows back to back (one batch entry in the tensor maps); N is the longest
+  // length.  Loads index from the sequence's first row; O rows are stored only
+  // up to the sequence end (plain stores for a tile the end falls inside), and
+  // the logsumexp of sequence b is [H, len_b] at lse + rowoff[b] * H.
+  const int* rowoff;
+  int T;
+  void* o;
+  long long o_rs, o_hs;  // element strides of O's rows and heads
 };
 constexpr unsigned kMapQ = 1, kMapK = 2, kMapV = 4, kMapO = 8;
 // Arguments of the decode instantiation (split-KV only).  The g query heads
@@ -200,7 +210,20 @@ __global__ void __launch_bounds__(384, 1)
   const int b = bh / p.H, h = bh % p.H;
   const int kvh = b * p.Hkv + h / p.g;
   const int q0 = pair * 256;
-  const int Lb = p.seqlens ? max(0, min(p.seqlens[b], p.N)) : p.N;  // valid rows of this batch entry
+  int Lb = p.seqlens ? max(0, min(p.seqlens[b], p.N)) : p.N;  // valid rows of this batch entry
+  // Tensor-map coordinates of this unit: first row, batch entry, head and kv head.
+  int rb = 0, cb = b, cbh = bh, ckvh = kvh;
+  bool packed = false;
+  if constexpr (kStrided) {
+    if (p.rowoff) {  // offsets clamped to the tensors' rows whatever they hold
+      packed = true;
+      rb = min(max(p.rowoff[b], 0), p.T);
+      Lb = min(min(max(p.rowoff[b + 1], rb), p.T) - rb, p.N);
+      cb = 0;
+      cbh = h;
+      ckvh = h / p.g;
+    }
+  }
   // Valid keys and the position of query row 0 (decode: Nk keys, queries are
   // the newest rows; otherwise the same rows as the queries, position 0).
   int Lk = Lb, qoff = 0;
@@ -289,8 +312,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < 2; ++t)
           for (int c = 0; c < C::kChunks; ++c)
             if constexpr (kStrided)
-              tma_load_tile(&tmQ, p.map4 & kMapQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128,
-                            bh, h, b);
+              tma_load_tile(&tmQ, p.map4 & kMapQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64,
+                            rb + q0 + t * 128, cbh, h, cb);
             else
               tma_load_3d(&tmQ, q_full, sQ + t * C::kTileBytes + c * 16384, c * 64, q0 + t * 128, bh);
       }
@@ -309,7 +332,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided)
               tma_load_tile(m, p.map4 & (which == 0 ? kMapK : kMapV), &kv_full[s], sKV + s * C::kTileBytes + c * 16384,
-                            c * 64, kv0, kvh, h / p.g, b);
+                            c * 64, rb + kv0, ckvh, h / p.g, cb);
             else
               tma_load_3d(m, &kv_full[s], sKV + s * C::kTileBytes + c * 16384, c * 64, kv0, kvh);
           }
@@ -530,6 +553,12 @@ __global__ void __launch_bounds__(384, 1)
       if (pad_row) l = 0.f;
       const float inv = (lb > 0.f && !pad_row) ? 1.f / lb : 0.f;
       uint8_t* sO = sQ + t * C::kTileBytes;  // Q_t is no longer read
+      // packed: the sequence ends inside this tile, so each valid row is stored by its own thread
+      __nv_bfloat16* orow = nullptr;
+      if constexpr (kStrided)
+        if (packed && tq0 + 128 > Lb && qrow < Lb)
+          orow = static_cast<__nv_bfloat16*>(p.o) + static_cast<long long>(rb + qrow) * p.o_rs +
+                 static_cast<long long>(h) * p.o_hs;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
@@ -550,19 +579,27 @@ __global__ void __launch_bounds__(384, 1)
           val.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv, __uint_as_float(o[8 * u + 7]) * inv);
           const uint32_t off = chunk * 16384 + r * 128 + (((u0 + u) ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(sO + off) = val;
+          if (kStrided && orow) *reinterpret_cast<uint4*>(orow + c + 8 * u) = val;
         }
       }
-      if (qrow < p.N)
-        p.lse[static_cast<size_t>(bh) * p.N + qrow] = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      const float lse_v = (l > 0.f) ? (m_used + log2f(l)) * kLn2 : -INFINITY;
+      if (packed) {
+        if (qrow < Lb) p.lse[static_cast<size_t>(rb) * p.H + static_cast<size_t>(h) * Lb + qrow] = lse_v;
+      } else if (qrow < p.N) {
+        p.lse[static_cast<size_t>(bh) * p.N + qrow] = lse_v;
+      }
       fence_proxy_async_smem();
     }
     // Every thread arrives (even after an abort) so the storing thread's
     // bounded wait below cannot be left short of arrivals by a live peer.
     mbar_arrive(&epi_bar[t]);
-    if (ok && r == 0 && tq0 < p.N && mbar_wait(&epi_bar[t], 0, abort_flag)) {
+    // packed: only whole tiles go through the TMA unit (its stores clip at the
+    // tensor's end, not at the sequence's)
+    const bool tma_out = packed ? tq0 + 128 <= Lb : tq0 < p.N;
+    if (ok && r == 0 && tma_out && mbar_wait(&epi_bar[t], 0, abort_flag)) {
       for (int c = 0; c < C::kChunks; ++c) {
         if constexpr (kStrided)
-          tma_store_tile(&tmO, p.map4 & kMapO, sQ + t * C::kTileBytes + c * 16384, c * 64, tq0, bh, h, b);
+          tma_store_tile(&tmO, p.map4 & kMapO, sQ + t * C::kTileBytes + c * 16384, c * 64, rb + tq0, cbh, h, cb);
         else
           tma_store_3d(&tmO, sQ + t * C::kTileBytes + c * 16384, c * 64, tq0, bh);
       }

@@ -203,31 +203,39 @@ fa_status fa_bwd_strided(const void* q, const void* k, const void* v, const void
 /*
  * Packed variable lengths: B sequences concatenated along the token axis, no
  * padding.  cu_seqlens: HOST pointer to B + 1 non-decreasing int32 offsets
- * with cu_seqlens[0] = 0; sequence b occupies token rows [cu_seqlens[b],
- * cu_seqlens[b+1]) of
+ * with cu_seqlens[0] = 0 (validated, and used to size the launch);
+ * cu_seqlens_dev: DEVICE pointer (16-byte aligned) to the same B + 1 values,
+ * read by the kernels, so it must stay unchanged until the stream has run the
+ * call (the fp32 path reads only the host copy and accepts NULL here; the
+ * kernels clamp every offset to [0, T], so differing copies give wrong values,
+ * never an access outside the tensors).  Sequence b occupies token rows
+ * [cu_seqlens[b], cu_seqlens[b+1]) of
  *   q, o, dout, dq   [T, H, d]     (T = cu_seqlens[B], d contiguous)
  *   k, v, dk, dv     [T, Hkv, d]
  *   lse              float; sequence b's [H, len_b] block starts at element
  *                    H * cu_seqlens[b]
  * Each sequence is its own attention problem (causal / window relative to its
  * first token; "FlashAttention" guide page, "Tiling through SRAM": padding and
- * lengths only alter how the tiles are laid out, not what is computed).  Every sequence runs as a
- * separate one-entry launch of the strided path on `stream` (the offsets are
- * read on the host), so very many short sequences pay one launch each; empty
- * sequences launch nothing.  fa_bwd_packed's workspace: at least
- * fa_bwd_packed_workspace_size(cu_seqlens, B, H, d, dtype) bytes (it is reused
+ * lengths only alter how the tiles are laid out, not what is computed).  bf16:
+ * one launch of each kernel covers every sequence; tiles start at each
+ * sequence's first row, and output rows are written only up to its end.  fp32:
+ * one launch per sequence (empty sequences launch nothing).  fa_bwd_packed's
+ * workspace: at least fa_bwd_packed_workspace_size(cu_seqlens, B, H, d, dtype)
+ * bytes -- for bf16 every sequence's rows padded to whole 128-row tiles plus
+ * 128 rows per sequence, per head; for fp32 the longest sequence's (reused
  * sequence after sequence, in stream order).  Errors: FA_ERR_INVALID_ARG for a
- * null pointer, B < 1, cu_seqlens[0] != 0 or decreasing offsets; otherwise as
- * fa_fwd / fa_bwd (with N the longest sequence).
+ * null or (bf16) missing / misaligned device offsets pointer, B < 1,
+ * cu_seqlens[0] != 0, decreasing offsets or T + 128 (B + 1) >= 2^30 (bf16);
+ * otherwise as fa_fwd / fa_bwd (with N the longest sequence).
  */
 fa_status fa_fwd_packed(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
-                        int B, int H, int Hkv, int d, float scale, int causal, int window, fa_dtype dtype,
-                        void* stream);
+                        const int* cu_seqlens_dev, int B, int H, int Hkv, int d, float scale, int causal, int window,
+                        fa_dtype dtype, void* stream);
 size_t fa_bwd_packed_workspace_size(const int* cu_seqlens, int B, int H, int d, fa_dtype dtype);
 fa_status fa_bwd_packed(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                        const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens, void* workspace,
-                        size_t ws_bytes, int B, int H, int Hkv, int d, float scale, int causal, int window,
-                        fa_dtype dtype, void* stream);
+                        const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens,
+                        const int* cu_seqlens_dev, void* workspace, size_t ws_bytes, int B, int H, int Hkv, int d,
+                        float scale, int causal, int window, fa_dtype dtype, void* stream);
 
 /*
  * Bytes of device workspace fa_bwd needs for these sizes (fp32 row terms

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.fa_version() == 100
+    assert L.fa_version() == 101
     for code in range(7):
         assert L.fa_status_string(code)
     assert L.fa_status_string(99) == b"unknown status"
@@ -252,7 +252,8 @@ def test_packed_rejects_bad_arguments(L):
     def fwd(offsets, B, **kw):
         a = dict(q=A, H=4, Hkv=2, d=128, dtype=0)
         a.update(kw)
-        return L.fa_fwd_packed(a["q"], A, A, A, A, offsets, B, a["H"], a["Hkv"], a["d"], f, 1, -1, a["dtype"], None)
+        return L.fa_fwd_packed(a["q"], A, A, A, A, offsets, a.get("dev", A), B, a["H"], a["Hkv"], a["d"], f, 1, -1,
+                               a["dtype"], None)
 
     assert fwd(None, 2) == 1
     assert fwd(cu(1, 5, 9), 2) == 1          # first offset must be 0
@@ -261,10 +262,18 @@ def test_packed_rejects_bad_arguments(L):
     assert fwd(cu(0, 5, 9), 2, H=3) == 1     # H % Hkv
     assert fwd(cu(0, 5, 9), 2, d=96) == 2
     assert fwd(cu(0, 5, 9), 2, q=A + 8) == 3
+    assert fwd(cu(0, 5, 9), 2, dev=None) == 1      # bf16 reads the offsets on the device
+    assert fwd(cu(0, 5, 9), 2, dev=A + 4) == 1     # ... from a 16-byte aligned copy
+    assert fwd(cu(0, 0, 0), 2) == 0                # no tokens: nothing to launch
+    # bf16: every sequence's rows in whole 128-row tiles at 128-aligned starts,
+    # 128 * (ceil(T / 128) + B) rows per head; fp32: the longest sequence
     need = L.fa_bwd_packed_workspace_size(cu(0, 300, 301, 1000), 3, 4, 128, 0)
-    assert need == L.fa_bwd_workspace_size(1, 4, 699, 128, 0)  # the longest sequence
+    assert need == L.fa_bwd_workspace_size(1, 4, 128 * (8 + 3), 128, 0)
+    assert L.fa_bwd_packed_workspace_size(cu(0, 300, 301, 1000), 3, 4, 128, 1) == \
+        L.fa_bwd_workspace_size(1, 4, 699, 128, 1)
     assert L.fa_bwd_packed_workspace_size(cu(0, 5, 4), 2, 4, 128, 0) == 0
-    assert L.fa_bwd_packed(*([A] * 9), cu(0, 300, 301, 1000), A, need - 1, 3, 4, 2, 128, f, 1, -1, 0, None) == 4
+    assert L.fa_bwd_packed(*([A] * 9), cu(0, 300, 301, 1000), A, A, need - 1, 3, 4, 2, 128, f, 1, -1, 0,
+                           None) == 4
 
 
 def test_seqlens_helper_rejects_copies():

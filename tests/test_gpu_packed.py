@@ -96,3 +96,63 @@ def test_packed_equals_padded_lengths_bitwise():
         assert torch.equal(l1[H * cu[b]:H * cu[b + 1]].view(H, L), l2[b, :, :L])
         assert torch.equal(g1[1][seg].transpose(0, 1), g2[1][b, :, :L])
         assert torch.equal(g1[2][seg].transpose(0, 1), g2[2][b, :, :L])
+
+
+def _short_lens(n, hi, seed):
+    """n sequence lengths in [0, hi], seeded, with a few empty and one-token ones."""
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, hi + 1, size=n).tolist()
+    lens[0], lens[n // 2], lens[-1] = 0, 1, hi
+    return lens
+
+
+@pytest.mark.parametrize("d,causal,window", [(64, True, -1), (128, False, -1), (64, False, 40)])
+def test_many_short_sequences_in_one_launch(d, causal, window):
+    """Hundreds of short sequences (tiles that end inside a sequence, empty and
+    one-token sequences, sequences that start mid-tile) against the oracle,
+    sequence by sequence, with the offsets handed over as a CUDA tensor."""
+    lens, H, Hkv = _short_lens(300, 200, 83 + d), 2, 1
+    q, k, v, do = packed_inputs(lens, H, Hkv, d, "bf16", 84)
+    cu = offsets(lens)
+    cu_dev = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    scale = 1.0 / d ** 0.5
+    o, lse = fa.fwd_packed(q.cuda(), k.cuda(), v.cuda(), cu_dev, scale, causal, window)
+    dq, dk, dv = fa.bwd_packed(q.cuda(), k.cuda(), v.cuda(), o, lse, do.cuda(), cu_dev, scale, causal, window)
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    o, lse, dq, dk, dv = (t.cpu() for t in (o, lse, dq, dk, dv))
+    for b, L in enumerate(lens):
+        if L == 0:
+            continue
+        sl = slice(cu[b], cu[b + 1])
+        as4 = lambda t: t[sl].transpose(0, 1).unsqueeze(0)  # noqa: E731  [1, heads, L, d]
+        want_o, want_l = ref.forward(as4(q), as4(k), as4(v), scale, causal, window)
+        gq, gk, gv = ref.backward(as4(q), as4(k), as4(v), as4(do), scale, causal, window)
+        compare("O", np64(as4(o)), want_o, "bf16")
+        compare("LSE", np64(lse[H * cu[b]:H * cu[b + 1]].view(1, H, L)), want_l, "bf16")
+        compare("dQ", np64(as4(dq)), gq, "bf16")
+        compare("dK", np64(as4(dk)), gk, "bf16")
+        compare("dV", np64(as4(dv)), gv, "bf16")
+
+
+def test_packed_writes_nothing_outside_its_rows():
+    """Outputs sit inside larger buffers holding a sentinel: rows before the
+    first token and after the last one (and the logsumexp around its T * H
+    values) must keep it, whichever way a tile's rows are stored."""
+    lens, H, Hkv, d, pad = [5, 130, 0, 257, 1, 77], 2, 1, 128, 300
+    q, k, v, do = (t.cuda() for t in packed_inputs(lens, H, Hkv, d, "bf16", 85))
+    cu = offsets(lens)
+    T = cu[-1]
+    sent = -7.0
+    big = lambda heads: torch.full((T + 2 * pad, heads, d), sent, dtype=torch.bfloat16, device="cuda")  # noqa: E731
+    ob, dqb, dkb, dvb = big(H), big(H), big(Hkv), big(Hkv)
+    lb = torch.full((T * H + 2 * 1024,), sent, dtype=torch.float32, device="cuda")
+    mid = slice(pad, pad + T)
+    o, lse = fa.fwd_packed(q, k, v, cu, causal=True, out=ob[mid], lse=lb[1024:1024 + T * H])
+    fa.bwd_packed(q, k, v, o, lse, do, cu, causal=True, grads=(dqb[mid], dkb[mid], dvb[mid]))
+    torch.cuda.synchronize()
+    assert fa.device_status() == 0
+    for name, t in (("O", ob), ("dQ", dqb), ("dK", dkb), ("dV", dvb)):
+        assert bool((t[:pad] == sent).all()) and bool((t[pad + T:] == sent).all()), name
+        assert bool(torch.isfinite(t[mid].float()).all()), name
+    assert bool((lb[:1024] == sent).all()) and bool((lb[1024 + T * H:] == sent).all())
