@@ -488,26 +488,31 @@ def _host_offsets(cu_seqlens):
     return (ctypes.c_int * len(vals))(*vals), len(vals) - 1
 
 
-def _device_offsets(cu_seqlens, host, B, device):
-    """Device int32 copy of the offsets that the kernels read: the caller's
-    tensor itself when it already is one (contiguous int32 on `device`),
-    otherwise a new tensor made from the host values on the current stream
-    (the calls run on that stream, after the copy)."""
+def _device_offsets(cu_seqlens, host, B, device, cu_seqlens_dev=None):
+    """Device int32 copy of the offsets that the kernels read: cu_seqlens_dev
+    when given, else the caller's tensor itself when it already is one
+    (contiguous int32 on `device`), otherwise a new tensor made from the host
+    values on the current stream (the calls run on that stream, after the copy)."""
     import torch
-    if isinstance(cu_seqlens, torch.Tensor) and cu_seqlens.is_cuda:
-        if cu_seqlens.device != device or cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_contiguous():
-            raise TypeError("a CUDA cu_seqlens must be a contiguous int32 tensor on q's device")
-        return cu_seqlens
+    t = cu_seqlens_dev if cu_seqlens_dev is not None else cu_seqlens
+    if isinstance(t, torch.Tensor) and t.is_cuda:
+        if t.device != device or t.dtype != torch.int32 or not t.is_contiguous() or t.numel() != B + 1:
+            raise TypeError("device offsets must be a contiguous int32 tensor of B + 1 values on q's device")
+        return t
+    if cu_seqlens_dev is not None:
+        raise TypeError("cu_seqlens_dev must be a CUDA int32 tensor")
     return torch.tensor([host[i] for i in range(B + 1)], dtype=torch.int32, device=device)
 
 
 def fwd_packed(q, k, v, cu_seqlens, scale: float | None = None, causal: bool = False, window: int = -1,
-               out=None, lse=None):
+               out=None, lse=None, cu_seqlens_dev=None):
     """O [T,H,d] and LSE (flat: sequence b's [H, len_b] block at H * cu[b]) for
     sequences packed along the token axis: q [T,H,d], k/v [T,Hkv,d], cu_seqlens
-    the B + 1 offsets (list, CPU tensor, or int32 tensor on q's device).  bf16
-    runs every sequence in one launch per kernel, reading a device copy of the
-    offsets."""
+    the B + 1 offsets (list, CPU tensor, or int32 tensor on q's device, which
+    is then read back to the host).  bf16 runs every sequence in one launch
+    per kernel, reading a device copy of the offsets: cu_seqlens_dev (an int32
+    tensor on q's device holding the same values) when given, else one made
+    here."""
     import torch
     if q.dim() != 3 or k.dim() != 3:
         raise ValueError("q, k, v must be 3-D [tokens, heads, head_dim]")
@@ -524,7 +529,7 @@ def fwd_packed(q, k, v, cu_seqlens, scale: float | None = None, causal: bool = F
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty(T * H, dtype=torch.float32, device=q.device) if lse is None else lse
-    cu_dev = _device_offsets(cu_seqlens, cu, B, q.device)
+    cu_dev = _device_offsets(cu_seqlens, cu, B, q.device, cu_seqlens_dev)
     code = _on(q.device, lib().fa_fwd_packed, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), cu,
                cu_dev.data_ptr(), B, H, Hkv, d, float(scale), int(bool(causal)), int(window), _dtype_code(q),
                _stream_ptr(q.device))
@@ -533,7 +538,7 @@ def fwd_packed(q, k, v, cu_seqlens, scale: float | None = None, causal: bool = F
 
 
 def bwd_packed(q, k, v, o, lse, do, cu_seqlens, scale: float | None = None, causal: bool = False, window: int = -1,
-               workspace=None, grads=None):
+               workspace=None, grads=None, cu_seqlens_dev=None):
     """bwd() of fwd_packed()."""
     import torch
     if q.dim() != 3 or k.dim() != 3:
@@ -554,7 +559,7 @@ def bwd_packed(q, k, v, o, lse, do, cu_seqlens, scale: float | None = None, caus
     need = int(lib().fa_bwd_packed_workspace_size(cu, B, H, d, code_t))
     ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq, dk, dv = grads if grads is not None else (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
-    cu_dev = _device_offsets(cu_seqlens, cu, B, q.device)
+    cu_dev = _device_offsets(cu_seqlens, cu, B, q.device, cu_seqlens_dev)
     code = _on(q.device, lib().fa_bwd_packed, q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu, cu_dev.data_ptr(), ws.data_ptr(),
                ws.numel(), B, H, Hkv, d, float(scale), int(bool(causal)), int(window), code_t,

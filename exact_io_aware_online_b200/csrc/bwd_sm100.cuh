@@ -31,8 +31,8 @@
 //   warp 15     TMA producer of the dO tiles
 // Registers: 128 per thread at launch; the fourth warpgroup drops to 96, the
 // compute warpgroups rise to 136 and the drain to 144 (136 + 136 + 144 + 96 =
-// 4 * 128, checked below), so a drain thread holds a whole dQ row and releases
-// the TMEM tile at once.
+// 4 * 128, checked below; strided instantiations 128 + 128 + 160 + 96), so a
+// drain thread holds a whole dQ row and releases the TMEM tile at once.
 //
 // dQ reduction.  Every (key tile, query tile) pair adds a 128 x D fp32 partial
 // into the global accumulator.  The drain loads the partial from TMEM into
@@ -105,6 +105,10 @@ struct BwdStridedParams : BwdParams {
   void* dk;
   void* dv;
   long long kv_rs, kv_hs;  // element strides of dK / dV rows and heads
+  // Packed, no window: a sequence's first key tile reaches every one of its
+  // query tiles and its job runs first in its slot, so that job stores its dQ
+  // partials instead of adding them, and the accumulator needs no zeroing.
+  int dq_first_store;
 };
 // First workspace row of packed sequence b (a multiple of 128): consecutive
 // sequences' padded row ranges [start, start + 128 * ceil(len / 128)) never
@@ -117,15 +121,22 @@ __device__ __forceinline__ void packed_range(const BwdStridedParams& p, int b, i
   len = min(min(max(p.rowoff[b + 1], rb), p.T) - rb, p.N);
 }
 // The packed sequence whose workspace rows hold row R (0 <= R < tp): the last b
-// with packed_ws_row(b) <= R (binary search; starts increase with b).
+// with packed_ws_row(b) <= R (starts increase with b).  Called by a whole warp
+// with the same R: each round the 32 lanes probe 32 evenly spaced candidates
+// and a ballot narrows the range 32-fold, so 1000 sequences take two rounds of
+// loads instead of ten dependent ones.
 __device__ __forceinline__ int packed_seq_of_ws_row(const BwdStridedParams& p, int R) {
+  const int lane = threadIdx.x & 31;
   int lo = 0, hi = p.B - 1;
   while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (packed_ws_row(min(max(p.rowoff[mid], 0), p.T), mid) <= R)
-      lo = mid;
-    else
-      hi = mid - 1;
+    const int step = (hi - lo + 32) / 32;  // ceil((hi - lo + 1) / 32)
+    const int idx = lo + lane * step;
+    const bool le = idx <= hi && packed_ws_row(min(max(p.rowoff[idx], 0), p.T), idx) <= R;
+    const int k = __popc(__ballot_sync(0xffffffffu, le));  // probes at or before R: lanes 0 .. k - 1
+    if (k == 0) break;  // R before every start (offsets that do not start at 0): sequence lo
+    const int nlo = lo + (k - 1) * step;
+    hi = min(hi, lo + k * step - 1);
+    lo = nlo;
   }
   return lo;
 }
@@ -170,8 +181,13 @@ static_assert(BwdCfg<128>::kSmemBytes <= 232448 && BwdCfg<64>::kSmemBytes <= 232
 // Per-thread register budgets after setmaxnreg (compute, compute, drain, MMA +
 // producers): an increase waits until decreases have freed the registers, so
 // the four must add up to the 4 x 128 the 512-thread launch provides.
-constexpr int kBwdRegsCompute = 136, kBwdRegsDrain = 144, kBwdRegsOther = 96;
-static_assert(2 * kBwdRegsCompute + kBwdRegsDrain + kBwdRegsOther == 4 * 128, "register split must sum to the launch");
+// The strided instantiations give the drain more: its epilogue also addresses
+// rows itself (packed sequences that end inside a key tile).
+template <bool kStrided>
+struct BwdRegs {
+  static constexpr int kCompute = kStrided ? 128 : 136, kDrain = kStrided ? 160 : 144, kOther = 96;
+  static_assert(2 * kCompute + kDrain + kOther == 4 * 128, "register split must sum to the launch");
+};
 
 // ---------------------------------------------------------------- preprocess
 // Half a warp per row (16 lanes x 16 bytes of O and of dO for D = 128, two rows
@@ -192,6 +208,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p)
   if constexpr (kStrided)
     if (packed) rows = static_cast<size_t>(p.H) * p.tp;
   const size_t row0 = (static_cast<size_t>(blockIdx.x) * 8 + warp) * kPreRowsPerWarp;
+  // packed: the block's 32 rows lie in one 128-row tile, so in one sequence
+  // (found once, by every warp as a whole)
+  int pb = 0;
+  if constexpr (kStrided)
+    if (packed) pb = packed_seq_of_ws_row(p, static_cast<int>((static_cast<size_t>(blockIdx.x) * 32) % p.tp));
 #pragma unroll
   for (int pass = 0; pass < kPreRowsPerWarp / kRowsPerPass; ++pass) {
     const size_t row = row0 + pass * kRowsPerPass + sub;  // over the workspace rows
@@ -202,13 +223,19 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p)
     if constexpr (kStrided) {
       if (packed && in) {
         const int h = static_cast<int>(row / p.tp), R = static_cast<int>(row % p.tp);
-        const int b = packed_seq_of_ws_row(p, R);
+        const int b = pb;
         packed_range(p, b, rb, len);
         n = R - packed_ws_row(rb, b);
         bh = static_cast<size_t>(b) * p.H + h;
       }
     }
-    if (in) {  // zero D floats of the dQ accumulator (every float is zeroed once, whatever the layout)
+    // Zero D floats of the dQ accumulator: linear rows 128t .. 128t + 127 cover
+    // exactly the floats of its 128-row tile t, whatever the order inside the
+    // tile.  Packed: tiles of a sequence's gap rows are never touched again.
+    bool zero = in;
+    if constexpr (kStrided)
+      if (packed) zero = in && !p.dq_first_store && n >= 0 && n / 128 * 128 < len;
+    if (zero) {
       float4* acc = reinterpret_cast<float4*>(p.dqacc + row * D);
       acc[2 * part] = make_float4(0.f, 0.f, 0.f, 0.f);
       acc[2 * part + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -294,6 +321,7 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs<kStrided> p) 
     }
   }
   if (!packed) nvalid = valid_rows(p, static_cast<int>(bh / p.H));
+  if (packed && (nbase < 0 || nbase >= nend)) return;  // gap rows: nothing to convert
   const int t128 = g >> 2, r0 = (g & 3) * 32;  // 128-row tile and first row inside it
 #pragma unroll
   for (int c = 0; c < D / 32; ++c) {  // 32 rows x 8 units of one chunk: 256 float4, one per thread
@@ -428,13 +456,43 @@ __global__ void __launch_bounds__(512, 1)
     slot = rem / gsz;
     bkv = g0 + rem % gsz;
   };
-  auto job_next = [&](Job J) {
+  bool packed = false;
+  if constexpr (kStrided) packed = p.rowoff != nullptr;
+  // Packed (one slot per sequence and kv head): the slot's key tiles one after
+  // another, j = sub, so the sequence's Q, dO and dQ accumulator tiles stay in
+  // L2 between its jobs.
+  auto tile_of = [&](Job J, int slot) {
+    return packed ? J.sub : (p.pairs ? (J.sub == 0 ? slot : p.ntiles - 1 - slot) : slot);
+  };
+  auto job_step = [&](Job J) {
     int slot, bkv;
     slot_of(J.gs, slot, bkv);
-    if (J.sub == 0 && p.pairs && p.ntiles - 1 - slot != slot) return Job{J.gs, 1};
+    if (packed ? J.sub + 1 < p.ntiles : (J.sub == 0 && p.pairs && p.ntiles - 1 - slot != slot))
+      return Job{J.gs, J.sub + 1};
     return Job{J.gs + static_cast<int>(gridDim.x), 0};
   };
-  const Job job0{static_cast<int>(blockIdx.x), 0};
+  // Packed: a key tile past its sequence's end is no job at all (its rows
+  // belong to the next sequence, so nothing is stored for it).
+  auto job_skip = [&](Job J) {
+    if constexpr (kStrided) {
+      if (packed) {
+        int slot, bkv, rb, len;
+        slot_of(J.gs, slot, bkv);
+        const int j = tile_of(J, slot);
+        packed_range(p, bkv / p.Hkv, rb, len);
+        return j * 128 >= len;
+      }
+    }
+    return false;
+  };
+  auto job_next = [&](Job J) {
+    do {
+      J = job_step(J);
+    } while (J.gs < nslots && job_skip(J));
+    return J;
+  };
+  Job job0{static_cast<int>(blockIdx.x), 0};
+  if (job0.gs < nslots && job_skip(job0)) job0 = job_next(job0);
   // One job: key tile j of kv head bkv, its query-tile range [ilo, ihi] and the
   // number of (query head, query tile) work items.  Work items are walked in
   // increasing order, skipping blocks a block-sparse mask switches off; every
@@ -447,8 +505,6 @@ __global__ void __launch_bounds__(512, 1)
     int rb, cb, ckv, cq0;     // tensor-map coordinates: first row, batch entry, kv head, first query head
     size_t w0;                // workspace row of (first query head, row 0); query head hq adds hq * wstride
   };
-  bool packed = false;
-  if constexpr (kStrided) packed = p.rowoff != nullptr;
   size_t wstride = p.Np;  // workspace rows per query head
   if constexpr (kStrided)
     if (packed) wstride = p.tp;
@@ -494,7 +550,7 @@ __global__ void __launch_bounds__(512, 1)
         U.w0 = static_cast<size_t>(U.kh * p.g) * p.tp + packed_ws_row(U.rb, U.b);
       }
     }
-    U.j = p.pairs ? (J.sub == 0 ? slot : p.ntiles - 1 - slot) : slot;
+    U.j = tile_of(J, slot);
     U.k0 = U.j * 128;
     U.ilo = 0;
     U.ihi = (max(U.Lb, 1) - 1) / 128;  // query tiles holding valid rows
@@ -559,7 +615,7 @@ __global__ void __launch_bounds__(512, 1)
 #endif
 
   if (warp >= 12) {
-    regs_dec<kBwdRegsOther>();
+    regs_dec<BwdRegs<kStrided>::kOther>();
     if (warp == 13 && lane == 0) {
       // ---------------------------------------------------------- producer: K, V, Q + LSE + D
       prefetch_tmap(&tmQ);
@@ -767,7 +823,7 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ P and dS
-    regs_inc<kBwdRegsCompute>();
+    regs_inc<BwdRegs<kStrided>::kCompute>();
     // Warpgroup w handles query columns [64w, 64w + 64); one key row per thread.
     const int w = warp >> 2, wl = warp & 3;
     const int r = wl * 32 + lane;
@@ -883,7 +939,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ drain and the dK/dV epilogue
-    regs_inc<kBwdRegsDrain>();
+    regs_inc<BwdRegs<kStrided>::kDrain>();
     const int wl = warp & 3;
     const int r = wl * 32 + lane;  // query row of the dQ tile (drain), key row (epilogue)
     const uint32_t lane_off = static_cast<uint32_t>(wl * 32) << 16;
@@ -893,6 +949,8 @@ __global__ void __launch_bounds__(512, 1)
     int git = 0, u = 0;
     for (Job J = job0; ok && J.gs < nslots; J = job_next(J), ++u) {
       const Unit U = unit(J);
+      bool first_store = false;  // this job writes the first dQ partial of each of its tiles
+      if constexpr (kStrided) first_store = packed && p.dq_first_store && U.j == 0;
       QCursor cur = first(U);
       for (int it = 0; it < U.total; ++it, cur = advance(U, cur)) {
         const int g = git + it;
@@ -925,7 +983,11 @@ __global__ void __launch_bounds__(512, 1)
           fence_proxy_async_smem();
           named_bar_sync(kBarDrain, 128);
           if (r == 0) {
-            bulk_reduce_add_f32(p.dqacc + ((tile0 + cur.i) * (D / 32) + c) * 4096, buf, C::kDqChunkBytes);
+            float* dst = p.dqacc + ((tile0 + cur.i) * (D / 32) + c) * 4096;
+            if (first_store)
+              bulk_store(dst, buf, C::kDqChunkBytes);
+            else
+              bulk_reduce_add_f32(dst, buf, C::kDqChunkBytes);
             bulk_commit();
           }
         }
@@ -937,7 +999,14 @@ __global__ void __launch_bounds__(512, 1)
       ok = named_bar_and(kBarDrainAnd, 128, mbar_wait(kv_done, u & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      if (r == 0) bulk_wait_read0();  // staging buffers no longer read by earlier reductions
+      // staging buffers no longer read by earlier reductions (first-store job:
+      // its stores complete, before the next jobs add into the same tiles)
+      if (r == 0) {
+        if (first_store)
+          bulk_wait0();
+        else
+          bulk_wait_read0();
+      }
       named_bar_sync(kBarDrain, 128);
       uint8_t* sDV = sDQ;                                  // bf16 128 x D tile in the TMA layout
       uint8_t* sDK = sDQ + (D == 128 ? 0 : C::kTileBytes);  // after dV's store has read it (D = 128)

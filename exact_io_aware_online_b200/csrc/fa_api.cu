@@ -496,8 +496,9 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
   p.causal = causal ? 1 : 0;
   p.window = window;
   p.ntiles = p.Np / 128;
-  p.pairs = (causal && window < 0) ? 1 : 0;
-  p.slots = p.pairs ? (p.ntiles + 1) / 2 : p.ntiles;
+  p.pairs = (causal && window < 0 && !pk) ? 1 : 0;
+  // packed: one slot per (sequence, kv head) holding all its key tiles
+  p.slots = pk ? 1 : (p.pairs ? (p.ntiles + 1) / 2 : p.ntiles);
   p.bmask = bmask;
   p.bmask_hs = bmask_hs;
   p.seqlens = seqlens;
@@ -544,6 +545,7 @@ fa_status bwd_bf16(const void* q, const void* k, const void* v, const void* o, c
       ps.rowoff = pk->rowoff;
       ps.T = pk->T;
       ps.tp = tp;
+      ps.dq_first_store = window < 0 ? 1 : 0;
       ps.dk = dk;
       ps.dv = dv;
       ps.kv_rs = lay.dk.n;

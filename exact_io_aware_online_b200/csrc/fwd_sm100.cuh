@@ -259,6 +259,9 @@ __global__ void __launch_bounds__(384, 1)
       while (j <= jhi && !block_on(0, j) && !block_on(1, j)) ++j;
     return j;
   };
+  // Packed: a unit past its sequence's end has nothing to compute or store (its
+  // rows belong to the next sequence): the whole CTA leaves before any setup.
+  if (packed && q0 >= Lb) return;
   int nkv = max(0, jhi - jlo + 1);
   if (qlast < q0) nkv = 0;  // the whole pair is padding
   if (kMask && nkv > 0) {
