@@ -21,7 +21,9 @@ def L():
 def test_header_declares_expected_entry_points():
     names = fa.exported_names()
     for n in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_last_device_status", "fa_status_string",
-              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_strided", "fa_bwd_strided", "fa_fwd_decode", "fa_fwd_packed", "fa_bwd_packed"):
+              "fa_version", "fa_set_timing_events", "fa_fwd_splitkv", "fa_fwd_splitkv_workspace_size", "fa_fwd_blocksparse", "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_strided", "fa_bwd_strided", "fa_fwd_decode", "fa_fwd_packed", "fa_bwd_packed",
+              "fa_fwd_decode_workspace_size", "fa_bwd_packed_workspace_size", "fa_bwd_noalloc",
+              "fa_debug_set_wait_limit", "fa_debug_set_stall"):
         assert n in names
 
 
