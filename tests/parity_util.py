@@ -82,11 +82,12 @@ def gpu_run(w: W.Workload, inputs: dict, device="cuda"):
     return dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv)
 
 
-def oracle_groups(w: W.Workload, inputs: dict, groups):
+def oracle_groups(w: W.Workload, inputs: dict, groups, row_block: int = 2048):
     """Oracle outputs for whole GQA groups: groups = [(b, kv_head), ...].
 
     Returns {(b, kh): dict(o, lse, dq [g heads], dk, dv)} computed from the
-    exact same (bf16-rounded) values the GPU saw.
+    exact same (bf16-rounded) values the GPU saw.  row_block: the oracle's row
+    blocking (it changes no value; small blocks keep a narrow band cheap).
     """
     g = w.H // w.Hkv
     out = {}
@@ -96,8 +97,8 @@ def oracle_groups(w: W.Workload, inputs: dict, groups):
         do = inputs["do"][b:b + 1, hs]
         k = inputs["k"][b:b + 1, kh:kh + 1]
         v = inputs["v"][b:b + 1, kh:kh + 1]
-        o, lse = ref.forward(q, k, v, w.scale, w.causal, w.window)
-        dq, dk, dv = ref.backward(q, k, v, do, w.scale, w.causal, w.window)
+        o, lse = ref.forward(q, k, v, w.scale, w.causal, w.window, row_block=row_block)
+        dq, dk, dv = ref.backward(q, k, v, do, w.scale, w.causal, w.window, row_block=row_block)
         out[(b, kh)] = dict(o=o[0], lse=lse[0], dq=dq[0], dk=dk[0, 0], dv=dv[0, 0])
     return out
 

@@ -150,3 +150,18 @@ def test_nothing_written_outside_outputs(dtype):
     for buf, _ in [(ob, o), (lb, lse)] + bufs:
         assert (buf[:pad] == -7777.0).all() and (buf[-pad:] == -7777.0).all()
     assert fa.device_status() == 0
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_long_sequence_narrow_window_every_element(causal):
+    """A sequence of 2^18 tokens (2048 key tiles per head, over ten jobs per CTA
+    of the persistent backward) with a narrow window, so the banded oracle
+    checks every element in seconds: row, tile and workspace indices at the
+    largest sizes the tests reach."""
+    w = _case("n262144_window48_d64", 1, 2, 1, 1 << 18, 64, "bf16", causal, 48, seed=12)
+    x = W.make_inputs(w)
+    got = gpu_run(w, x)
+    t0 = time.perf_counter()
+    want = oracle_groups(w, x, _all_groups(w), row_block=256)
+    worst = check_groups(w, got, want)
+    print(w.name, "causal" if causal else "", worst, f"oracle {time.perf_counter() - t0:.1f} s")
