@@ -284,12 +284,14 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdArgs<kStrided> p)
 // one bulk reduce-add covers it).  Inside a chunk, row r holds its 32 floats in
 // eight 16-byte units, unit u stored at position u ^ (r % 8): the drain's
 // shared-memory writes (one row per thread) then spread over all banks.
-// Element (n, c) of head bh sits at float index
-//   dqacc_chunk(bh, ntiles, n / 128, c / 32) + (n % 128) * 32
+// Tiles are numbered by workspace row / 128 (head bh's rows start at row
+// bh * Np, or for packed sequences at h * tp + the sequence's start).  Element
+// (row n, column c) sits at float index
+//   dqacc_chunk<D>(n / 128, c / 32) + (n % 128) * 32
 //     + (((c % 32) / 4) ^ (n % 8)) * 4 + c % 4.
 template <int D>
-__device__ __forceinline__ size_t dqacc_chunk(size_t bh, int ntiles, int tile, int chunk) {
-  return ((bh * static_cast<size_t>(ntiles) + tile) * (D / 32) + chunk) * 4096;
+__device__ __forceinline__ size_t dqacc_chunk(size_t tile, int chunk) {
+  return (tile * (D / 32) + chunk) * 4096;
 }
 
 // ---------------------------------------------------------------- dQ convert
@@ -327,7 +329,7 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const BwdArgs<kStrided> p) 
   for (int c = 0; c < D / 32; ++c) {  // 32 rows x 8 units of one chunk: 256 float4, one per thread
     const int rr = threadIdx.x >> 3, up = threadIdx.x & 7;
     const int u = up ^ (rr & 7);  // r0 is a multiple of 8, so (r0 + rr) % 8 = rr % 8
-    const float4 a = reinterpret_cast<const float4*>(p.dqacc + ((tile0 + t128) * (D / 32) + c) * 4096 +
+    const float4 a = reinterpret_cast<const float4*>(p.dqacc + dqacc_chunk<D>(tile0 + t128, c) +
                                                      static_cast<size_t>(r0) * 32)[threadIdx.x];
     *reinterpret_cast<float4*>(&tile[rr][c * 32 + 4 * u]) = a;
   }
@@ -967,7 +969,7 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_before();
         mbar_arrive(dq_empty);  // TMEM tile free before the reductions are staged
         if (r == 0) FA_TRACE_AT(4, g, 1);
-        // the accumulator's 128-row tiles of this query head (dqacc_chunk's order)
+        // the accumulator's first 128-row tile of this query head
         const size_t tile0 = (U.w0 + cur.hq * wstride) / 128;
 #pragma unroll
         for (int c = 0; c < C::kDqChunks; ++c, ++nchunk) {
@@ -983,7 +985,7 @@ __global__ void __launch_bounds__(512, 1)
           fence_proxy_async_smem();
           named_bar_sync(kBarDrain, 128);
           if (r == 0) {
-            float* dst = p.dqacc + ((tile0 + cur.i) * (D / 32) + c) * 4096;
+            float* dst = p.dqacc + dqacc_chunk<D>(tile0 + cur.i, c);
             if (first_store)
               bulk_store(dst, buf, C::kDqChunkBytes);
             else
