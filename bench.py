@@ -51,15 +51,24 @@ KERNEL_SOURCES = {  # the files each profiled kernel (and its launch configurati
 }
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and with whitespace runs collapsed: edits to
+    comments alone leave the compiled kernel, and so the hash, unchanged."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(kernel: str | None = None) -> str:
-    """Hash of the sources of `kernel` (of every CUDA source when None)."""
+    """Hash of the code (comments dropped) of the sources of `kernel` (of every
+    CUDA source when None)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_online_b200", "csrc")
     names = KERNEL_SOURCES.get(kernel) if kernel else None
     for name in sorted(names or os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode())
-            h.update(f.read())
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

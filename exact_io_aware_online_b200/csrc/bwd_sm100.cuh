@@ -74,9 +74,9 @@ struct BwdParams {
   int causal, window;
   int ntiles;  // Np / 128
   int group;   // kv heads per rasterisation group (kept L2-resident together)
-  int slots;   // CTAs per kv head
-  int pairs;   // 1 (causal): ceil(ntiles / 2) CTAs, each running key tiles j and ntiles - 1 - j;
-               // 0: ntiles CTAs, one key tile each
+  int slots;   // slots (units of work the CTAs take in turn) per kv head
+  int pairs;   // 1 (causal): ceil(ntiles / 2) slots, each holding key tiles j and ntiles - 1 - j;
+               // 0: ntiles slots of one key tile each (packed: one slot of every key tile)
   // block-sparse mode (non-null bmask): 0/1 per 128 x 128 block, [query block]
   // [key block] per query head, bmask_hs elements apart (0: shared by all heads)
   const uint8_t* bmask;
