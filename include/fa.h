@@ -252,8 +252,9 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d, fa_dtype dtype);
  * kv head sum over its H / Hkv query heads.  workspace: caller-owned device
  * memory of at least fa_bwd_workspace_size() bytes, 16-byte aligned; its
  * contents on entry do not matter and are garbage on return.  dk, dv, o and
- * lse are deterministic; dq (bf16 path) sums tile contributions with atomics,
- * so its last bits may vary from run to run.
+ * lse are deterministic; dq (bf16 path) adds the tile contributions in L2 in
+ * whatever order they arrive (TMA bulk reduce-adds), so its last bits may vary
+ * from run to run.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
