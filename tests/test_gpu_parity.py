@@ -165,3 +165,16 @@ def test_long_sequence_narrow_window_every_element(causal):
     want = oracle_groups(w, x, _all_groups(w), row_block=256)
     worst = check_groups(w, got, want)
     print(w.name, "causal" if causal else "", worst, f"oracle {time.perf_counter() - t0:.1f} s")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_many_short_heads_sampled_groups(causal):
+    """B=64, 32 query heads on 8 kv heads, N=200: 512 kv heads of short jobs
+    spread over the persistent backward's CTAs and the forward's head groups;
+    the first, a middle and the last kv groups against the oracle."""
+    w = _case("b64_h32kv8_n200_d128", 64, 32, 8, 200, 128, "bf16", causal, -1, seed=13)
+    x = W.make_inputs(w)
+    got = gpu_run(w, x)
+    groups = [(0, 0), (31, 5), (63, 7)]
+    worst = check_groups(w, got, oracle_groups(w, x, groups))
+    print(w.name, "causal" if causal else "", worst)
