@@ -73,8 +73,17 @@ def test_algorithmic_bytes_and_ridge_side():
 
 def test_bench_rejects_bad_option_combinations():
     """Host-side option checks run before anything touches a GPU."""
-    for extra in (["--warmup", "2"], ["--decode", "1", "--impl", "reference"]):
+    for extra in (["--warmup", "2"], ["--decode", "1", "--impl", "reference"], ["--packed", "10", "--impl", "reference"]):
         out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *extra], capture_output=True,
                              text=True, timeout=300, cwd=ROOT)
         assert out.returncode != 0
-        assert "warmup" in out.stderr or "--decode" in out.stderr, out.stderr[-500:]
+        assert any(w in out.stderr for w in ("warmup", "--decode", "--packed")), out.stderr[-500:]
+
+
+def test_packed_workload_lengths_are_seeded_and_in_range():
+    sys.path.insert(0, ROOT)
+    import bench
+    a, b = bench.packed_lengths(1000), bench.packed_lengths(1000)
+    assert a == b and len(a) == 1000
+    lo, hi = bench.PACKED_SHAPE["lo"], bench.PACKED_SHAPE["hi"]
+    assert min(a) >= lo and max(a) <= hi and abs(sum(a) / len(a) - (lo + hi) / 2) < 10
