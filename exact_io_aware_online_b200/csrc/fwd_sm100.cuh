@@ -116,7 +116,14 @@ struct FwdCfg {
   static constexpr int kStages = (D == 128) ? 4 : 8;
   static constexpr int kSmemQ = 2 * kTileBytes;
   static constexpr int kSmemKV = kStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 9;
+  static constexpr int kNumBars = 1 + 2 * kStages + 15;
+  // P_t V is issued in kPvParts key ranges, each as soon as the softmax threads
+  // have stored that range of P_t, so only the last range (and the next Q K^T)
+  // sits between the end of the exponentials and the next score tile.  Two
+  // halves pay at D = 64 (forward 5% faster at B=4 H=16 N=2048); at D = 128
+  // the extra store wait in the exponent loop costs what the earlier half
+  // saves (measured: equal or slower), so one range.
+  static constexpr int kPvParts = (D == 64) ? 2 : 1;
   static constexpr int kSmemBytes = 1024 + kSmemQ + kSmemKV + 8 * kNumBars + 16;
   static constexpr int kThreads = 384;
   static constexpr uint32_t kTmemCols = 512;
@@ -133,9 +140,9 @@ constexpr float kLn2 = 0.69314718055994530942f;
 // bf16 in four 32-key chunks; accumulates the fp32 row sum (l) and the sum of
 // the bf16-rounded values (lb).  kPoly: one pair in four uses exp2_poly2 so
 // the special-function unit is not the only source of exponentials.
-template <bool kPoly>
+template <bool kPoly, int kParts>
 __device__ __forceinline__ void exp_row_to_tmem(const float (&s)[128], float sl2, float ms, uint32_t tS, float& l,
-                                                float& lb) {
+                                                float& lb, uint64_t* part_bar) {
   const uint64_t sl2x2 = f2(sl2, sl2), nmsx2 = f2(-ms, -ms);
   // Row sums on packed fp32 pairs, two independent accumulators each.  rs:
   // exact fp32 weights (gives the logsumexp); rsb: the bf16-rounded weights
@@ -161,6 +168,11 @@ __device__ __forceinline__ void exp_row_to_tmem(const float (&s)[128], float sl2
       rsb2[u & 1] = fadd2(rsb2[u & 1], f2(__uint_as_float(pk[u] << 16), __uint_as_float(pk[u] & 0xffff0000u)));
     }
     tmem_st16(tS + ch * 16, pk);
+    if (kParts > 1 && ch < 3 && (ch + 1) % (4 / kParts) == 0) {  // this key range of P is in TMEM
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&part_bar[(ch + 1) / (4 / kParts) - 1]);
+    }
   }
   float a0, a1, b0, b1;
   f2_split(fadd2(rs2[0], rs2[1]), a0, a1);
@@ -189,6 +201,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* o_full = s_full + 4;
   uint64_t* epi_bar = s_full + 6;  // softmax threads -> storing thread: O tile staged
   uint64_t* mma_idle = s_full + 8;  // every product the MMA thread issued has completed
+  uint64_t* p_part = s_full + 9;    // [t * 3 + i]: softmax -> MMA, key range i of P_t stored (i < kPvParts - 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -278,6 +291,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
+      for (int i = 0; i < 3; ++i) mbar_init(&p_part[3 * t + i], 128);
       mbar_init(&o_full[t], 1);
       mbar_init(&epi_bar[t], 128);
     }
@@ -359,11 +373,21 @@ __global__ void __launch_bounds__(384, 1)
                   sdesc_sw128(aKV + slot * C::kTileBytes + off, 16, 1024), kIdescS, k > 0);
         }
       };
-      auto pv = [&](int t, int slot, bool acc) {  // O_t += P_t V
+      // O_t += P_t V, each key range issued once its part of P_t is stored
+      // (false: the wait gave up).
+      auto pv = [&](int t, int slot, bool acc, uint32_t parity, int tj) {
+        constexpr int kStep = 8 / C::kPvParts;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-          umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8,
-                  sdesc_sw128(aKV + slot * C::kTileBytes + k * 2048, 16384, 1024), kIdescO, acc || k > 0);
+        for (int i = 0; i < C::kPvParts; ++i) {
+          if (!mbar_wait(i + 1 < C::kPvParts ? &p_part[3 * t + i] : &p_full[t], parity, abort_flag)) return false;
+          FA_TRACE_AT(2 + t, tj, i);
+          tc_fence_after();
+#pragma unroll
+          for (int k = i * kStep; k < (i + 1) * kStep; ++k)
+            umma_ts(tmem + 256 + t * D, tmem + t * 128 + k * 8,
+                    sdesc_sw128(aKV + slot * C::kTileBytes + k * 2048, 16384, 1024), kIdescO, acc || k > 0);
+        }
+        return true;
       };
       bool ok = nkv > 0 && mbar_wait(q_full, 0, abort_flag);
       // decode: a second query tile of padding rows only gets no products
@@ -373,21 +397,14 @@ __global__ void __launch_bounds__(384, 1)
       for (int jj = 0; ok && jj < nkv; ++jj, it += 2) {
         const int sK = it % C::kStages;
         if (!(ok = mbar_wait(&kv_full[sK], (it / C::kStages) & 1, abort_flag))) break;
+        FA_TRACE_AT(4, jj, 0);
         tc_fence_after();
         const int sVprev = (it - 1 + C::kStages) % C::kStages;
-        if (jj > 0) {
-          if (!(ok = mbar_wait(&p_full[0], (jj - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          pv(0, sVprev, jj > 1);
-        }
+        if (jj > 0 && !(ok = pv(0, sVprev, jj > 1, (jj - 1) & 1, jj - 1))) break;
         qk(0, sK);
         umma_commit(&s_full[0]);
         if (jj > 0) {
-          if (has1) {
-            if (!(ok = mbar_wait(&p_full[1], (jj - 1) & 1, abort_flag))) break;
-            tc_fence_after();
-            pv(1, sVprev, jj > 1);
-          }
+          if (has1 && !(ok = pv(1, sVprev, jj > 1, (jj - 1) & 1, jj - 1))) break;
           umma_commit(&kv_empty[sVprev]);
         }
         if (has1) {
@@ -397,14 +414,13 @@ __global__ void __launch_bounds__(384, 1)
         umma_commit(&kv_empty[sK]);
         const int sV = (it + 1) % C::kStages;
         if (!(ok = mbar_wait(&kv_full[sV], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+        FA_TRACE_AT(4, jj, 1);
         tc_fence_after();
       }
       if (ok) {
         const int sV = (it - 1) % C::kStages;
         for (int t = 0; t < (has1 ? 2 : 1) && ok; ++t) {
-          if (!(ok = mbar_wait(&p_full[t], (nkv - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          pv(t, sV, nkv > 1);
+          if (!(ok = pv(t, sV, nkv > 1, (nkv - 1) & 1, nkv - 1))) break;
           umma_commit(&o_full[t]);
         }
       }
@@ -454,6 +470,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int ch = 0; ch < 4; ++ch) tmem_st16(tS + ch * 16, z);
         tmem_wait_st();
         tc_fence_before();
+        for (int i = 0; i + 1 < C::kPvParts; ++i) mbar_arrive(&p_part[3 * t + i]);
         mbar_arrive(&p_full[t]);
         continue;
       }
@@ -461,6 +478,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[c * 32]));
       tmem_wait_ld();
+      if (lane == 0 && wl == 0) FA_TRACE_AT(t, jj, 2);
       float s[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sraw[c]);
@@ -481,13 +499,17 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = static_cast<uint32_t>(c - c_lo) <= span ? s[c] : -INFINITY;
       }
-      float mx8[8];  // eight independent partial maxima (short dependency chains)
+      // Eight independent partial maxima (short dependency chains): mx8[i] covers
+      // columns i, i + 8, ..., i + 120.
+      float mx8[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+      for (int i = 0; i < 8; ++i) mx8[i] = fmax3(s[i], s[8 + i], s[16 + i]);
 #pragma unroll
-      for (int c = 8; c < 128; c += 16)
+      for (int c = 24; c < 120; c += 16)
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = fmax3(mx8[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx8[i] = fmaxf(mx8[i], s[120 + i]);
       const float mx = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]), fmaxf(fmax3(mx8[3], mx8[4], mx8[5]), fmax3(mx8[6], mx8[7], mx8[7])));
       const float m_new = fmaxf(m_used, mx * sl2);
       bool need = false;
@@ -515,10 +537,11 @@ __global__ void __launch_bounds__(384, 1)
         tmem_wait_st();
       }
       const float ms = (m_used == -INFINITY) ? 0.f : m_used;
+      if (lane == 0 && wl == 0) FA_TRACE_AT(t, jj, 3);
       if (full && C::kPolyExp)
-        exp_row_to_tmem<true>(s, sl2, ms, tS, l, lb);
+        exp_row_to_tmem<true, C::kPvParts>(s, sl2, ms, tS, l, lb, p_part + 3 * t);
       else
-        exp_row_to_tmem<false>(s, sl2, ms, tS, l, lb);
+        exp_row_to_tmem<false, C::kPvParts>(s, sl2, ms, tS, l, lb, p_part + 3 * t);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[t]);

@@ -8,13 +8,15 @@ head for the two workloads whose oracle takes about a minute.
 """
 import time
 
+import numpy as np
 import pytest
 import torch
 
 import exact_io_aware_online_b200 as fa
 from exact_io_aware_online_b200 import workloads as W
 
-from parity_util import check_groups, gpu_run, oracle_groups
+from parity_util import check_groups, compare, gpu_run, np64, oracle_groups
+from oracle import ref
 
 pytestmark = pytest.mark.gpu
 
@@ -178,3 +180,28 @@ def test_many_short_heads_sampled_groups(causal):
     groups = [(0, 0), (31, 5), (63, 7)]
     worst = check_groups(w, got, oracle_groups(w, x, groups))
     print(w.name, "causal" if causal else "", worst)
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_dominant_key_at_every_column(d):
+    """Row r's largest score (about 100 above the others, natural units) sits
+    at column r mod 128 of a 128-key tile (and at r mod 64 + 64 for d = 64), so
+    every column position of a tile holds some row's dominant key.  The running
+    maximum has to see it wherever it is: weights taken against a maximum that
+    missed it would be 2^144 or more, past the fp32 range.  Forward outputs
+    only: with the dominant keys' weights summing to one, dQ is the small
+    remainder of terms of size |k| ~ 34 and reflects the bf16 rounding of O
+    (through D = rowsum(dO * O)) more than anything the forward computes."""
+    N, c = 256, 34.0
+    w = _case(f"dominant_d{d}", 1, 1, 1, N, d, "bf16", False, -1)
+    g = torch.Generator("cpu").manual_seed(5)
+    basis = torch.zeros(N, d)
+    basis[torch.arange(N), torch.arange(N) % d] = c
+    q = basis + 0.1 * torch.randn(N, d, generator=g)
+    k = basis + 0.1 * torch.randn(N, d, generator=g)
+    v = torch.randn(N, d, generator=g)
+    x = {n: t.view(1, 1, N, d).to(torch.bfloat16).contiguous() for n, t in (("q", q), ("k", k), ("v", v))}
+    o, lse = fa.fwd(*(x[n].cuda() for n in ("q", "k", "v")), w.scale, False, -1)
+    torch.cuda.synchronize()
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], w.scale, False, -1)
+    compare("O", np64(o)[0, 0], np.asarray(o_ref)[0, 0], "bf16")
+    compare("LSE", np64(lse)[0, 0], np.asarray(lse_ref)[0, 0], "bf16")
