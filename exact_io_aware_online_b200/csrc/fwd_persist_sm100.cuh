@@ -8,7 +8,8 @@
 //   - the next unit's Q loads as soon as this unit's last Q K^T has read sQ
 //     (barrier q_empty), so its first products follow this unit's last P V;
 //   - O is staged in a tile of its own (sO, one query tile at a time, handed
-//     on by barrier so_free) since sQ already holds the next unit's Q.
+//     on between the two query tiles by barriers so_free[t]) since sQ already
+//     holds the next unit's Q.
 // It pays where units are short (a few key tiles: narrow windows, short or
 // packed sequences), whose CTA start, first loads and epilogue would otherwise
 // take a large share of the time.  Dense and strided / packed layouts; no
@@ -23,7 +24,7 @@ template <int D>
 struct FwdPersistCfg {
   using C = FwdCfg<D>;
   static constexpr int kSmemO = C::kTileBytes;
-  static constexpr int kNumBars = C::kNumBars + 2;  // + q_empty, so_free
+  static constexpr int kNumBars = C::kNumBars + 3;  // + q_empty, so_free[2]
   static constexpr int kSmemBytes = 1024 + C::kSmemQ + C::kSmemKV + kSmemO + 8 * kNumBars + 16;
   static_assert(kSmemBytes <= 232448, "shared memory per CTA");
   // setmaxnreg split: the unit loop needs more than 72 registers in the
@@ -113,7 +114,13 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* mma_idle = s_full + 8;  // every product the MMA thread issued has completed
   uint64_t* p_part = s_full + 9;    // [t * 3 + i]: softmax -> MMA, key range i of P_t stored (i < kPvParts - 1)
   uint64_t* q_empty = s_full + 15;  // MMA -> producer: the unit's last Q K^T has read sQ
-  uint64_t* so_free = s_full + 16;  // storing thread -> softmax threads: the O store has read sO
+  // so_free[t]: the other query tile's storing thread -> tile t's softmax
+  // threads: its O store has read sO, so tile t may write its O there.  One
+  // barrier per direction, each with one arriving and one waiting tile: a
+  // tile cannot reach its next wait before the phase it waits for has begun
+  // (a single shared barrier let a tile whose own previous arrival was still
+  // pending take the older phase for the one it wanted).
+  uint64_t* so_free = s_full + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + PC::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -133,7 +140,8 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
-    mbar_init(so_free, 1);
+    mbar_init(&so_free[0], 1);
+    mbar_init(&so_free[1], 1);
     for (int i = 0; i < C::kStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
@@ -389,10 +397,11 @@ __global__ void __launch_bounds__(384, 1)
       kt += U.nkv;
       // ---------------------------------------------------------- epilogue
       if (U.nkv > 0) ok = mbar_wait(&o_full[t], uo & 1, abort_flag);
-      // sO is free once the previous tile's store (the other query tile's, or
-      // the previous unit's second) has read it
-      const int prev = 2 * ne + t - 1;
-      if (ok && prev >= 0) ok = mbar_wait(so_free, prev & 1, abort_flag);
+      // sO is free once the other query tile's previous store has read it:
+      // tile 1 waits for tile 0's store of this unit (so_free[1] completion ne),
+      // tile 0 for tile 1's store of the previous unit (so_free[0], ne - 1).
+      const int prev = t == 1 ? ne : ne - 1;
+      if (ok && prev >= 0) ok = mbar_wait(&so_free[t], prev & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (ok) {
         tc_fence_after();
@@ -443,7 +452,11 @@ __global__ void __launch_bounds__(384, 1)
       // tensor's end, not at the sequence's)
       const bool tma_out = U.packed ? tq0 + 128 <= U.Lb : tq0 < p.N;
       if (r == 0) {
-        if (ok && tma_out && mbar_wait(&epi_bar[t], ne & 1, abort_flag)) {
+        // Wait for every thread of the tile to have written sO, whether or not
+        // it is stored from there: the next wait on epi_bar[t] then finds this
+        // phase complete, and sO is released only once nobody writes it.
+        const bool staged = mbar_wait(&epi_bar[t], ne & 1, abort_flag);
+        if (ok && tma_out && staged) {
           for (int c = 0; c < C::kChunks; ++c) {
             if constexpr (kStrided)
               tma_store_tile(&tmO, p.map4 & kMapO, sO + c * 16384, c * 64, U.rb + tq0, U.cbh, U.h, U.cb);
@@ -453,7 +466,7 @@ __global__ void __launch_bounds__(384, 1)
           bulk_commit();
           bulk_wait_read0();
         }
-        mbar_arrive(so_free);  // sO may be rewritten
+        mbar_arrive(&so_free[1 - t]);  // the other tile may write sO
       }
       if (U.nkv > 0) ++uo;
       ++ne;

@@ -53,6 +53,8 @@ CASES = [
     ("bshd_full_d64", 2, 3, 3, 520, 64, "bf16", False, -1),
     ("bshd_window_d128", 1, 2, 1, 900, 128, "bf16", False, 100),
     ("bshd_fp32_d64", 2, 2, 1, 300, 64, "fp32", True, -1),
+    # more units than SMs, five key tiles each at most: the persistent forward on 4-D maps
+    ("bshd_many_units_causal_d128", 16, 8, 4, 1000, 128, "bf16", True, -1),
 ]
 
 

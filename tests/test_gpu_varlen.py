@@ -22,6 +22,14 @@ def _built():
         pytest.skip("no GPU")
 
 
+def _lens(n, hi, seed):
+    """Seeded lengths in [0, hi], the first three forced to 0, 1 and hi."""
+    g = torch.Generator().manual_seed(seed)
+    lens = torch.randint(0, hi + 1, (n,), generator=g).tolist()
+    lens[:3] = [0, 1, hi]
+    return lens
+
+
 CASES = [
     # name, B, H, Hkv, N, d, dtype, causal, window, lens
     ("causal_d128", 3, 2, 1, 700, 128, "bf16", True, -1, [700, 383, 1]),
@@ -29,6 +37,11 @@ CASES = [
     ("window_d128", 2, 2, 2, 900, 128, "bf16", False, 100, [900, 257]),
     ("zero_length", 2, 1, 1, 300, 64, "bf16", True, -1, [0, 300]),
     ("fp32_causal", 2, 2, 1, 300, 64, "fp32", True, -1, [300, 77]),
+    # Many short units (at most a few key tiles each, more units than SMs): the
+    # forward runs persistent CTAs over several units each, including padding
+    # pairs with no key tile (O = 0, LSE = -inf) and empty sequences.
+    ("many_units_causal_d64", 40, 8, 2, 700, 64, "bf16", True, -1, _lens(40, 700, 61)),
+    ("many_units_window_d128", 24, 4, 4, 1500, 128, "bf16", False, 64, _lens(24, 1500, 62)),
 ]
 
 
