@@ -47,7 +47,8 @@ def peaks():
 
 KERNEL_SOURCES = {  # the files each profiled kernel (and its launch configuration) is built from
     "bwd_sm100_kernel": ("bwd_sm100.cuh", "sm100_ptx.cuh", "layout.cuh", "fa_api.cu"),
-    "fwd_sm100_kernel": ("fwd_sm100.cuh", "fwd_persist_sm100.cuh", "sm100_ptx.cuh", "layout.cuh", "fa_api.cu"),
+    "fwd_sm100_kernel": ("fwd_sm100.cuh", "sm100_ptx.cuh", "layout.cuh", "fa_api.cu"),
+    "fwd_persist_kernel": ("fwd_persist_sm100.cuh", "fwd_sm100.cuh", "sm100_ptx.cuh", "layout.cuh", "fa_api.cu"),
 }
 
 
