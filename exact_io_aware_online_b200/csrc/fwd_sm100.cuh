@@ -7,7 +7,9 @@
 // Softmax"): the running maximum m, the running sum l and the unnormalised
 // accumulator O~, rescaled when the maximum moves (Step 3's merge with one new
 // block at a time).  Only O and the logsumexp reach global memory ("FlashAttention"
-// guide page, "Tiling through SRAM").
+// guide page, "Tiling through SRAM").  Where units are short (a few key tiles
+// each), fwd_persist_sm100.cuh runs the same tiles with CTAs that take unit
+// after unit.
 //
 // Roles (384 threads, three warpgroups):
 //   warps 0-3   softmax for query tile 0, one thread per row (TMEM lanes 0-127)
