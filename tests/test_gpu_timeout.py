@@ -24,12 +24,16 @@ LIMIT_NS = 20_000_000  # 20 ms instead of the default two seconds
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("d", [128, 64])
-def test_stalled_load_reports_timeout_then_recovers(d):
+@pytest.mark.parametrize("d,B,H", [(128, 1, 4), (64, 1, 4), (128, 40, 2)],
+                         ids=["d128", "d64", "d128_persistent_forward"])
+def test_stalled_load_reports_timeout_then_recovers(d, B, H):
+    """B=40 H=2: 160 short units (three key tiles at most) on fewer CTAs than
+    units, so the forward runs its persistent kernel and every role leaves
+    the unit loop on the abort."""
     if not torch.cuda.is_available():
         pytest.skip("no GPU")
     _build.build()
-    w = W.Workload(f"stall_d{d}", 1, 4, 2, 384, d, "bf16", True, -1, 31)
+    w = W.Workload(f"stall_d{d}_b{B}", B, H, H // 2, 384, d, "bf16", True, -1, 31)
     x = W.make_inputs(w)
     q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
     assert fa.device_status() == 0
@@ -49,5 +53,6 @@ def test_stalled_load_reports_timeout_then_recovers(d):
         fa.debug_set_wait_limit(0)
     assert fa.device_status() == 0  # the status word was cleared by the reads above
     got = gpu_run(w, x)  # asserts a clean status itself
-    want = oracle_groups(w, x, [(0, kh) for kh in range(w.Hkv)])
+    groups = [(b, kh) for b in sorted({0, w.B - 1}) for kh in range(w.Hkv)]
+    want = oracle_groups(w, x, groups)
     check_groups(w, got, want)
